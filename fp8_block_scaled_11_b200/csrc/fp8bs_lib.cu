@@ -1,0 +1,445 @@
+// fp8bs_lib.cu -- the C ABI declared in include/fp8bs.h: argument validation,
+// TMA tensor-map encoding, launch configuration, and the device error flag.
+// The kernels are in quant_kernels.cuh and gemm_kernel.cuh (one translation
+// unit, so the error flag is a plain __device__ variable).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fp8bs.h"
+#include "quant_kernels.cuh"
+#include "gemm_kernel.cuh"
+
+using namespace fp8bs;
+
+namespace {
+
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool sm100 = false;
+    int num_sms = 0;
+    int* err_ptr = nullptr;
+    bool gemm_attr_set[4] = {false, false, false, false};
+    int quant_blocks[10] = {0};  // resident CTAs per SM, per quant kernel kind
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+fp8bs_status get_device(DeviceInfo** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8BS_ERR_CUDA;
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!d.ready) {
+            int major = 0;
+            if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return FP8BS_ERR_CUDA;
+            d.sm100 = (major == 10);
+            if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FP8BS_ERR_CUDA;
+            if (d.sm100) {
+                void* p = nullptr;
+                if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return FP8BS_ERR_CUDA;
+                d.err_ptr = static_cast<int*>(p);
+            }
+            if (g_encode == nullptr) {
+                void* fn = nullptr;
+                cudaDriverEntryPointQueryResult q;
+                if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || fn == nullptr)
+                    return FP8BS_ERR_CUDA;
+                g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+            }
+            d.ready = true;
+        }
+    }
+    if (!d.sm100) return FP8BS_ERR_NO_SM100;
+    *out = &d;
+    return FP8BS_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t dtype_size(fp8bs_dtype t) { return t == FP8BS_F32 ? 4 : 2; }
+inline bool valid_dtype(fp8bs_dtype t) { return t == FP8BS_BF16 || t == FP8BS_F32; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+fp8bs_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? FP8BS_OK : FP8BS_ERR_CUDA;
+}
+
+// Persistent grid: resident CTAs per SM (occupancy calculator) x SMs, capped by the work.
+template <typename Kernel>
+int persistent_grid(DeviceInfo* d, int kind, Kernel k, int64_t work_ctas)
+{
+    if (d->quant_blocks[kind] == 0) {
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k, 256, 0) != cudaSuccess || nb < 1) nb = 1;
+        d->quant_blocks[kind] = nb;
+    }
+    const int64_t cap = (int64_t)d->quant_blocks[kind] * d->num_sms;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(cap, work_ctas));
+}
+
+// 2-D tensor map over a row-major matrix: inner dim `inner` elements, `outer`
+// rows, row pitch `pitch_bytes`, box {box_inner, box_outer}.
+fp8bs_status make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base, uint64_t inner,
+                      uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                      CUtensorMapSwizzle swz)
+{
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {pitch_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    (void)esize;
+    CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP8BS_OK : FP8BS_ERR_CUDA;
+}
+
+struct SplitPlan {
+    int tiles_m, tiles_n, splits;
+    int64_t ldw;
+    size_t ws_bytes;
+};
+
+SplitPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms)
+{
+    SplitPlan s;
+    s.tiles_m = (int)cdiv(M, kBM);
+    s.tiles_n = (int)cdiv(N, kBN);
+    const int64_t tiles = (int64_t)s.tiles_m * s.tiles_n;
+    const int64_t Kb = cdiv(K, kBK);
+    int splits = 1;
+    if (tiles * 2 <= num_sms) {
+        // fill the SMs, but keep >= 4 K-blocks per split so the pipeline runs
+        splits = (int)std::min<int64_t>(num_sms / tiles, std::max<int64_t>(1, Kb / 4));
+        splits = std::max(1, std::min(splits, 64));
+    }
+    s.splits = splits;
+    s.ldw = (N + 3) & ~int64_t(3);
+    s.ws_bytes = splits > 1 ? (size_t)splits * (size_t)M * (size_t)s.ldw * sizeof(float) : 0;
+    return s;
+}
+
+int num_sms_current()
+{
+    DeviceInfo* d = nullptr;
+    if (get_device(&d) != FP8BS_OK) return 148;
+    return d->num_sms;
+}
+
+template <int MODE>
+fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA,
+                                const CUtensorMap& tSB, const GemmParams& p, cudaStream_t stream)
+{
+    auto k = gemm_fp8_kernel<MODE>;
+    if (!d->gemm_attr_set[MODE]) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::alloc) != cudaSuccess)
+            return FP8BS_ERR_CUDA;
+        d->gemm_attr_set[MODE] = true;
+    }
+    const int grid = (int)std::min<int64_t>(p.num_units, d->num_sms);
+    k<<<grid, kThreads, SmemLayout::alloc, stream>>>(tA, tB, tSA, tSB, p);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fp8bs_status_string(fp8bs_status s)
+{
+    switch (s) {
+    case FP8BS_OK: return "FP8BS_OK";
+    case FP8BS_ERR_INVALID_ARG: return "FP8BS_ERR_INVALID_ARG";
+    case FP8BS_ERR_UNSUPPORTED: return "FP8BS_ERR_UNSUPPORTED";
+    case FP8BS_ERR_ALIGNMENT: return "FP8BS_ERR_ALIGNMENT";
+    case FP8BS_ERR_WORKSPACE: return "FP8BS_ERR_WORKSPACE";
+    case FP8BS_ERR_CUDA: return "FP8BS_ERR_CUDA";
+    case FP8BS_ERR_TIMEOUT: return "FP8BS_ERR_TIMEOUT";
+    case FP8BS_ERR_NO_SM100: return "FP8BS_ERR_NO_SM100";
+    }
+    return "FP8BS_UNKNOWN_STATUS";
+}
+
+fp8bs_status fp8bs_check_device_error(cudaStream_t stream)
+{
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return FP8BS_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return FP8BS_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return FP8BS_ERR_CUDA;
+        return FP8BS_ERR_TIMEOUT;
+    }
+    return FP8BS_OK;
+}
+
+// ---------------------------------------------------------------- quantization
+
+fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
+                             int64_t ldq, float* scale_inv, int64_t ld_scale, int transpose_out, cudaStream_t stream)
+{
+    if (!valid_dtype(xt)) return FP8BS_ERR_UNSUPPORTED;
+    if (x == nullptr || q == nullptr || scale_inv == nullptr || rows < 1 || cols < 1) return FP8BS_ERR_INVALID_ARG;
+    if (transpose_out != 0 && transpose_out != 1) return FP8BS_ERR_INVALID_ARG;
+    if (ldx < cols) return FP8BS_ERR_INVALID_ARG;
+    const int64_t out_rows = transpose_out ? cols : rows;
+    const int64_t out_cols = transpose_out ? rows : cols;
+    if (ldq < out_cols || ld_scale < out_rows) return FP8BS_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(scale_inv)) return FP8BS_ERR_ALIGNMENT;
+    if ((ldx * (int64_t)dtype_size(xt)) % 16 || ldq % 16 || ld_scale % 4 || cols % 16) return FP8BS_ERR_ALIGNMENT;
+    if (transpose_out && rows % 16) return FP8BS_ERR_ALIGNMENT;
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+
+    if (!transpose_out) {
+        const int64_t items = cdiv(rows, 32) * cdiv(cols, 128);
+        const int64_t ctas = cdiv(items, 8);
+        if (xt == FP8BS_BF16) {
+            auto k = quant_1x128_rows_kernel<__nv_bfloat16>;
+            int g = persistent_grid(d, 0, k, ctas);
+            k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
+        } else {
+            auto k = quant_1x128_rows_kernel<float>;
+            int g = persistent_grid(d, 1, k, ctas);
+            k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
+        }
+    } else {
+        const int64_t ctas = cdiv(rows, 128) * cdiv(cols, 64);
+        if (xt == FP8BS_BF16) {
+            auto k = quant_1x128_cols_kernel<__nv_bfloat16>;
+            int g = persistent_grid(d, 2, k, ctas);
+            k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
+        } else {
+            auto k = quant_1x128_cols_kernel<float>;
+            int g = persistent_grid(d, 3, k, ctas);
+            k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
+        }
+    }
+    return launch_status();
+}
+
+fp8bs_status fp8_quant_128x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
+                               int64_t ldq, float* scale_inv, int64_t ld_scale, uint8_t* q_t, int64_t ldq_t,
+                               float* scale_inv_t, int64_t ld_scale_t, cudaStream_t stream)
+{
+    if (!valid_dtype(xt)) return FP8BS_ERR_UNSUPPORTED;
+    if (x == nullptr || rows < 1 || cols < 1 || (q == nullptr && q_t == nullptr)) return FP8BS_ERR_INVALID_ARG;
+    if (ldx < cols) return FP8BS_ERR_INVALID_ARG;
+    const int64_t rb = cdiv(rows, 128), cb = cdiv(cols, 128);
+    if (q != nullptr) {
+        if (scale_inv == nullptr || ldq < cols || ld_scale < rb) return FP8BS_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(scale_inv) || ldq % 16 || ld_scale % 4) return FP8BS_ERR_ALIGNMENT;
+    }
+    if (q_t != nullptr) {
+        if (scale_inv_t == nullptr || ldq_t < rows || ld_scale_t < cb) return FP8BS_ERR_INVALID_ARG;
+        if (!aligned16(q_t) || !aligned16(scale_inv_t) || ldq_t % 16 || ld_scale_t % 4) return FP8BS_ERR_ALIGNMENT;
+    }
+    if (!aligned16(x) || (ldx * (int64_t)dtype_size(xt)) % 16 || rows % 16 || cols % 16) return FP8BS_ERR_ALIGNMENT;
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+    const int64_t ctas = rb * cb;
+    if (xt == FP8BS_BF16) {
+        auto k = quant_128x128_kernel<__nv_bfloat16>;
+        int g = persistent_grid(d, 4, k, ctas);
+        k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale,
+                                 q_t, ldq_t, scale_inv_t, ld_scale_t);
+    } else {
+        auto k = quant_128x128_kernel<float>;
+        int g = persistent_grid(d, 5, k, ctas);
+        k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale, q_t,
+                                 ldq_t, scale_inv_t, ld_scale_t);
+    }
+    return launch_status();
+}
+
+size_t fp8_quant_tensor_workspace_size(int64_t n)
+{
+    (void)n;
+    return (size_t)kTensorPartials * sizeof(float);
+}
+
+fp8bs_status fp8_quant_tensor(const void* x, fp8bs_dtype xt, int64_t n, uint8_t* q, float* scale_inv,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (!valid_dtype(xt)) return FP8BS_ERR_UNSUPPORTED;
+    if (x == nullptr || q == nullptr || scale_inv == nullptr || n < 1) return FP8BS_ERR_INVALID_ARG;
+    if (workspace == nullptr || workspace_bytes < fp8_quant_tensor_workspace_size(n)) return FP8BS_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(scale_inv) & 3) ||
+        n % 16)
+        return FP8BS_ERR_ALIGNMENT;
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+    const int64_t chunks = n / 8;
+    const int parts = (int)std::max<int64_t>(1, std::min<int64_t>(kTensorPartials, cdiv(chunks, 256 * 4)));
+    float* partial = static_cast<float*>(workspace);
+    if (xt == FP8BS_BF16) {
+        tensor_amax_kernel<__nv_bfloat16><<<parts, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), n, partial);
+        auto k = tensor_quant_kernel<__nv_bfloat16>;
+        int g = persistent_grid(d, 6, k, cdiv(chunks, 256));
+        k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), n, partial, parts, q, scale_inv);
+    } else {
+        tensor_amax_kernel<float><<<parts, 256, 0, stream>>>(static_cast<const float*>(x), n, partial);
+        auto k = tensor_quant_kernel<float>;
+        int g = persistent_grid(d, 7, k, cdiv(chunks, 256));
+        k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), n, partial, parts, q, scale_inv);
+    }
+    return launch_status();
+}
+
+fp8bs_status fp8_quant_rowwise(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
+                               int64_t ldq, float* scale_inv, cudaStream_t stream)
+{
+    if (!valid_dtype(xt)) return FP8BS_ERR_UNSUPPORTED;
+    if (x == nullptr || q == nullptr || scale_inv == nullptr || rows < 1 || cols < 1) return FP8BS_ERR_INVALID_ARG;
+    if (ldx < cols || ldq < cols) return FP8BS_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scale_inv) & 3) ||
+        (ldx * (int64_t)dtype_size(xt)) % 16 || ldq % 16 || cols % 16)
+        return FP8BS_ERR_ALIGNMENT;
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+    const int64_t ctas = cdiv(rows, 8);
+    if (xt == FP8BS_BF16) {
+        auto k = quant_rowwise_kernel<__nv_bfloat16>;
+        int g = persistent_grid(d, 8, k, ctas);
+        k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx, q, ldq, scale_inv);
+    } else {
+        auto k = quant_rowwise_kernel<float>;
+        int g = persistent_grid(d, 9, k, ctas);
+        k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ldx, q, ldq, scale_inv);
+    }
+    return launch_status();
+}
+
+// ---------------------------------------------------------------- GEMM
+
+size_t fp8_scaled_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8bs_scale_mode mode)
+{
+    (void)mode;
+    if (M < 1 || N < 1 || K < 1) return 0;
+    return plan_gemm(M, N, K, num_sms_current()).ws_bytes;
+}
+
+fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* Bt,
+                             int64_t ldb, const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
+                             fp8bs_scale_mode mode, fp8bs_scale_layout layout, void* D, int64_t ldd,
+                             fp8bs_dtype out_dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (mode < FP8BS_SCALE_TENSOR || mode > FP8BS_SCALE_BLOCK_1x128_1x128) return FP8BS_ERR_UNSUPPORTED;
+    if (layout != FP8BS_SCALE_COL_MAJOR || !valid_dtype(out_dtype)) return FP8BS_ERR_UNSUPPORTED;
+    if (A == nullptr || Bt == nullptr || scale_a == nullptr || scale_b == nullptr || D == nullptr) return FP8BS_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 16) return FP8BS_ERR_INVALID_ARG;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8BS_ERR_INVALID_ARG;
+    if (lda < K || ldb < K || ldd < N) return FP8BS_ERR_INVALID_ARG;
+    const int64_t Kb = cdiv(K, kBK), Nb = cdiv(N, 128);
+    const bool block = (mode == FP8BS_SCALE_BLOCK_1x128_128x128 || mode == FP8BS_SCALE_BLOCK_1x128_1x128);
+    if (block) {
+        if (ld_sa < M) return FP8BS_ERR_INVALID_ARG;
+        if (mode == FP8BS_SCALE_BLOCK_1x128_128x128 && ld_sb < Nb) return FP8BS_ERR_INVALID_ARG;
+        if (mode == FP8BS_SCALE_BLOCK_1x128_1x128 && ld_sb < N) return FP8BS_ERR_INVALID_ARG;
+        if (ld_sa % 4 || ld_sb % 4) return FP8BS_ERR_ALIGNMENT;
+    }
+    if (K % 16 || lda % 16 || ldb % 16 || (ldd * (int64_t)dtype_size(out_dtype)) % 16) return FP8BS_ERR_ALIGNMENT;
+    if (!aligned16(A) || !aligned16(Bt) || !aligned16(D) || !aligned16(scale_a) || !aligned16(scale_b))
+        return FP8BS_ERR_ALIGNMENT;
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+
+    SplitPlan plan = plan_gemm(M, N, K, d->num_sms);
+    if (plan.splits > 1) {
+        if (workspace == nullptr && workspace_bytes == 0) {
+            plan.splits = 1;                     // split-K disabled by the caller
+        } else if (workspace == nullptr || workspace_bytes < plan.ws_bytes) {
+            return FP8BS_ERR_WORKSPACE;
+        } else if (!aligned16(workspace)) {
+            return FP8BS_ERR_ALIGNMENT;
+        }
+    }
+
+    CUtensorMap tA, tB, tSA, tSB;
+    std::memset(&tSA, 0, sizeof tSA);
+    std::memset(&tSB, 0, sizeof tSB);
+    if ((st = make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, lda, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
+        return st;
+    if ((st = make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Bt, K, N, ldb, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
+        return st;
+    const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    switch (mode) {
+    case FP8BS_SCALE_TENSOR:
+        break;
+    case FP8BS_SCALE_ROWWISE:
+        if ((st = make_map(&tSA, f32, 4, scale_a, M, 1, (M * 4 + 15) & ~int64_t(15), kBM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        if ((st = make_map(&tSB, f32, 4, scale_b, N, 1, (N * 4 + 15) & ~int64_t(15), kBN, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        break;
+    case FP8BS_SCALE_BLOCK_1x128_128x128:
+        if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, kBM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        if ((st = make_map(&tSB, f32, 4, scale_b, Nb, Kb, ld_sb * 4, 4, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        break;
+    case FP8BS_SCALE_BLOCK_1x128_1x128:
+        if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, kBM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        if ((st = make_map(&tSB, f32, 4, scale_b, N, Kb, ld_sb * 4, kBN, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        break;
+    }
+
+    GemmParams p;
+    p.M = (int32_t)M;
+    p.N = (int32_t)N;
+    p.K = (int32_t)K;
+    p.Kb = (int32_t)Kb;
+    p.tiles_m = plan.tiles_m;
+    p.tiles_n = plan.tiles_n;
+    p.splits = plan.splits;
+    p.group_m = 16;
+    p.num_units = (int64_t)plan.tiles_m * plan.tiles_n * plan.splits;
+    p.D = D;
+    p.ldd = ldd;
+    p.out_f32 = out_dtype == FP8BS_F32;
+    p.ws = static_cast<float*>(workspace);
+    p.ldw = plan.ldw;
+    p.sa = scale_a;
+    p.sb = scale_b;
+    p.err = d->err_ptr;
+
+    switch (mode) {
+    case FP8BS_SCALE_TENSOR: st = launch_gemm<kModeTensor>(d, tA, tB, tSA, tSB, p, stream); break;
+    case FP8BS_SCALE_ROWWISE: st = launch_gemm<kModeRowwise>(d, tA, tB, tSA, tSB, p, stream); break;
+    case FP8BS_SCALE_BLOCK_1x128_128x128: st = launch_gemm<kModeBlock128>(d, tA, tB, tSA, tSB, p, stream); break;
+    case FP8BS_SCALE_BLOCK_1x128_1x128: st = launch_gemm<kModeBlock1x128>(d, tA, tB, tSA, tSB, p, stream); break;
+    }
+    if (st != FP8BS_OK) return st;
+    if (plan.splits > 1) {
+        const int64_t chunks = M * ((N + 3) / 4);
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(chunks, 256), (int64_t)d->num_sms * 8));
+        splitk_reduce_kernel<<<grid, 256, 0, stream>>>(p.ws, plan.splits, M, N, plan.ldw, D, ldd, p.out_f32);
+        st = launch_status();
+    }
+    return st;
+}
+
+}  // extern "C"

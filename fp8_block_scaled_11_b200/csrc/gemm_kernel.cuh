@@ -1,0 +1,446 @@
+// gemm_kernel.cuh -- FP8 (e4m3) scaled GEMM on the sm_100a tensor cores.
+//
+// Computes  D[m,n] = sum_kb rA(m,kb) * rB(n,kb) * P_kb[m,n],
+//           P_kb[m,n] = sum_{k in K-block kb} qA[m,k] * qB[n,k]
+// i.e. the dequantized matmul that pytorch/ao PR #4209 "[codex] add repro for
+// blockwise _scaled_mm investigation" (What Changed) uses as ground truth, for
+// the (1x128, 128x128) and (1x128, 1x128) recipes of that page and the
+// per-tensor / rowwise recipes of ROCm/aiter issue #1765 and pytorch/pytorch
+// issue #159940.
+//
+// Structure (one persistent CTA per SM, 320 threads = 10 warps):
+//   warp 0      TMA producer: for each K-block, one 128x128 tile of A and one
+//               256x128 tile of B (bytes, 128-byte swizzle) into an S-stage
+//               shared-memory ring; per-K-block scale vectors into a separate
+//               ring (they are consumed later, by the epilogue).
+//   warp 1      TMEM owner + MMA issuer: one elected thread issues four
+//               tcgen05.mma (128x256x32, e4m3 x e4m3 -> fp32) per K-block into
+//               one of two 256-column TMEM accumulators, and commits the smem
+//               stage back to the producer when the MMAs have read it.
+//   warps 2-9   epilogue / promotion: per accumulation group (one K-block for
+//               the block recipes; the whole K range for tensor/rowwise) they
+//               tcgen05.ld the partial sums, multiply by the scale product and
+//               add into fp32 registers (packed f32x2 FMA), then release the
+//               TMEM buffer so the MMA of group g+2 can start.  At the end of
+//               a tile the registers are converted and stored.
+// The per-K-block promotion keeps every partial sum in fp32 with the exact
+// scale product of its block, which is what makes any number of K blocks
+// (1000, 1001, 1002, ...) safe: scale indexing is kb*ld + i with no padding
+// or parity assumption.
+//
+// Every mbarrier wait is bounded (kWaitLimitNs).  A wait that runs out sets
+// the library error flag and a CTA-wide abort flag; all roles then leave their
+// loops, the producer waits (bounded) for its TMA copies in flight, the MMA
+// thread waits (bounded) for its MMAs in flight, and TMEM is freed before exit.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace fp8bs {
+
+constexpr int kBM = 128;             // tile rows (A rows, TMEM lanes)
+constexpr int kBN = 256;             // tile cols (B rows, TMEM columns per accumulator)
+constexpr int kBK = 128;             // K-block = scale block = one 128-byte swizzle row
+constexpr int kStages = 4;           // A/B smem ring depth
+constexpr int kScaleStages = 8;      // scale ring depth (>= kStages + 2 + 1)
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
+constexpr uint64_t kWaitLimitNs = 4000000000ull;   // pipeline waits
+constexpr uint64_t kDrainLimitNs = 1000000000ull;  // exit-time waits for work in flight
+
+constexpr uint32_t kATileBytes = kBM * kBK;            // 16 KB
+constexpr uint32_t kBTileBytes = kBN * kBK;            // 32 KB
+constexpr uint32_t kScaleEntryBytes = (kBM + kBN) * 4; // sa[128] then sb[256]
+
+struct SmemLayout {
+    static constexpr uint32_t a_off = 0;
+    static constexpr uint32_t b_off = a_off + kStages * kATileBytes;
+    static constexpr uint32_t sc_off = b_off + kStages * kBTileBytes;
+    static constexpr uint32_t bar_off = sc_off + kScaleStages * kScaleEntryBytes;
+    // barriers: ab_full[S], ab_empty[S], sc_full[SS], sc_empty[SS], tm_full[2], tm_empty[2], drain
+    static constexpr uint32_t n_bars = 2 * kStages + 2 * kScaleStages + 4 + 1;
+    static constexpr uint32_t misc_off = bar_off + n_bars * 8;
+    static constexpr uint32_t total = misc_off + 16;
+    static constexpr uint32_t alloc = total + 1024;     // slack to align the base to 1024 B
+};
+
+enum GemmMode : int { kModeTensor = 0, kModeRowwise = 1, kModeBlock128 = 2, kModeBlock1x128 = 3 };
+
+struct GemmParams {
+    int32_t M, N, K;
+    int32_t Kb;                 // number of K blocks
+    int32_t tiles_m, tiles_n;
+    int32_t splits;             // K splits per tile (1 = no split-K)
+    int32_t group_m;            // rasterization band height in tiles
+    int64_t num_units;          // tiles_m * tiles_n * splits
+    void* D;                    // output (bf16 or fp32) when splits == 1
+    int64_t ldd;
+    int32_t out_f32;
+    float* ws;                  // split-K partials [splits][M][ldw] fp32
+    int64_t ldw;
+    const float* sa;            // tensor mode: scale pointers read directly
+    const float* sb;
+    int* err;                   // library error flag
+};
+
+__device__ __forceinline__ void decode_unit(const GemmParams& p, int64_t u, int& tm, int& tn, int& kb0, int& kb1,
+                                            int& split)
+{
+    const int64_t tile = u / p.splits;
+    split = (int)(u - tile * p.splits);
+    // grouped rasterization: bands of group_m tile-rows, column-major inside a band
+    const int64_t band_tiles = (int64_t)p.group_m * p.tiles_n;
+    const int64_t band = tile / band_tiles;
+    const int64_t in_band = tile - band * band_tiles;
+    const int band_m0 = (int)(band * p.group_m);
+    const int band_h = min(p.group_m, p.tiles_m - band_m0);
+    tm = band_m0 + (int)(in_band % band_h);
+    tn = (int)(in_band / band_h);
+    kb0 = (int)(((int64_t)p.Kb * split) / p.splits);
+    kb1 = (int)(((int64_t)p.Kb * (split + 1)) / p.splits);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                const GemmParams p)
+{
+    constexpr bool kPromote = (MODE == kModeBlock128 || MODE == kModeBlock1x128);
+    constexpr bool kScaleRing = (MODE != kModeTensor);
+    constexpr bool kColScales = (MODE == kModeBlock1x128 || MODE == kModeRowwise);
+    constexpr uint32_t kScaleTx = kBM * 4 + (kColScales ? kBN * 4 : 16);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bars = sbase + SmemLayout::bar_off;
+    auto ab_full = [&](int s) { return bars + 8u * s; };
+    auto ab_empty = [&](int s) { return bars + 8u * (kStages + s); };
+    auto sc_full = [&](int s) { return bars + 8u * (2 * kStages + s); };
+    auto sc_empty = [&](int s) { return bars + 8u * (2 * kStages + kScaleStages + s); };
+    auto tm_full = [&](int b) { return bars + 8u * (2 * kStages + 2 * kScaleStages + b); };
+    auto tm_empty = [&](int b) { return bars + 8u * (2 * kStages + 2 * kScaleStages + 2 + b); };
+    const uint32_t drain_bar = bars + 8u * (2 * kStages + 2 * kScaleStages + 4);
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + SmemLayout::misc_off);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc_off + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(ab_full(s), 1);
+            mbar_init(ab_empty(s), 1);
+        }
+        for (int s = 0; s < kScaleStages; ++s) {
+            mbar_init(sc_full(s), 1);
+            mbar_init(sc_empty(s), kEpiWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tm_full(b), 1);
+            mbar_init(tm_empty(b), kEpiWarps);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        if (kScaleRing) {
+            prefetch_tensormap(&tmSA);
+            prefetch_tensormap(&tmSB);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(sbase + SmemLayout::misc_off, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        atomicOr(p.err, 1);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int ss = 0;
+            uint32_t sphase = 0;
+            bool ok = true;
+            // per stage: was it ever filled, and the parity of its latest fill
+            uint32_t filled = 0, fill_par = 0, sfilled = 0, sfill_par = 0;
+            auto issue_scales = [&](int m0, int n0, int kb) -> bool {
+                if (!mbar_wait_bounded(sc_empty(ss), sphase ^ 1u, abort_flag, kWaitLimitNs)) return false;
+                const uint32_t dst = sbase + SmemLayout::sc_off + ss * kScaleEntryBytes;
+                mbar_arrive_expect_tx(sc_full(ss), kScaleTx);
+                tma_load_2d(dst, &tmSA, sc_full(ss), m0, kb);
+                if (kColScales) {
+                    tma_load_2d(dst + kBM * 4, &tmSB, sc_full(ss), n0, kb);
+                } else {
+                    tma_load_2d(dst + kBM * 4, &tmSB, sc_full(ss), (n0 / 128) & ~3, kb);
+                }
+                sfilled |= 1u << ss;
+                sfill_par = (sfill_par & ~(1u << ss)) | (sphase << ss);
+                if (++ss == kScaleStages) { ss = 0; sphase ^= 1u; }
+                return true;
+            };
+            for (int64_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                int tm, tn, kb0, kb1, split;
+                decode_unit(p, u, tm, tn, kb0, kb1, split);
+                const int m0 = tm * kBM, n0 = tn * kBN;
+                if (MODE == kModeRowwise) ok = issue_scales(m0, n0, 0);
+                for (int kb = kb0; kb < kb1 && ok; ++kb) {
+                    if (!mbar_wait_bounded(ab_empty(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    mbar_arrive_expect_tx(ab_full(stage), kATileBytes + kBTileBytes);
+                    tma_load_2d(sbase + SmemLayout::a_off + stage * kATileBytes, &tmA, ab_full(stage), kb * kBK, m0);
+                    tma_load_2d(sbase + SmemLayout::b_off + stage * kBTileBytes, &tmB, ab_full(stage), kb * kBK, n0);
+                    filled |= 1u << stage;
+                    fill_par = (fill_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (kPromote) ok = issue_scales(m0, n0, kb);
+                }
+            }
+            if (!ok) give_up();
+            // drain: every issued TMA copy must have landed before the CTA exits
+            for (int s = 0; s < kStages; ++s)
+                if (filled >> s & 1u) mbar_wait_bounded(ab_full(s), fill_par >> s & 1u, nullptr, kDrainLimitNs);
+            for (int s = 0; s < kScaleStages; ++s)
+                if (sfilled >> s & 1u) mbar_wait_bounded(sc_full(s), sfill_par >> s & 1u, nullptr, kDrainLimitNs);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_e4m3_f32(kBM, kBN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int tb = 0;
+            uint32_t tphase = 0;
+            bool ok = true, issued = false;
+            for (int64_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                int tm, tn, kb0, kb1, split;
+                decode_unit(p, u, tm, tn, kb0, kb1, split);
+                const int ngroups = kPromote ? (kb1 - kb0) : 1;
+                int kb = kb0;
+                for (int g = 0; g < ngroups && ok; ++g) {
+                    const int kb_end = kPromote ? kb + 1 : kb1;
+                    if (!mbar_wait_bounded(tm_empty(tb), tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(tb * kBN);
+                    for (; kb < kb_end; ++kb) {
+                        if (!mbar_wait_bounded(ab_full(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t a_addr = sbase + SmemLayout::a_off + stage * kATileBytes;
+                        const uint32_t b_addr = sbase + SmemLayout::b_off + stage * kBTileBytes;
+#pragma unroll
+                        for (int k = 0; k < kBK / 32; ++k) {
+                            const uint64_t adesc = smem_desc_k_sw128(a_addr + k * 32);
+                            const uint64_t bdesc = smem_desc_k_sw128(b_addr + k * 32);
+                            const uint32_t acc = (kPromote ? (k > 0) : (kb > kb0 || k > 0)) ? 1u : 0u;
+                            umma_f8(d_tmem, adesc, bdesc, idesc, acc);
+                        }
+                        issued = true;
+                        umma_commit(ab_empty(stage));
+                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    }
+                    if (!ok) break;
+                    umma_commit(tm_full(tb));
+                    if (++tb == 2) { tb = 0; tphase ^= 1u; }
+                }
+            }
+            if (!ok) give_up();
+            if (issued) {
+                // all MMAs of this thread complete before TMEM can be freed
+                umma_commit(drain_bar);
+                mbar_wait_bounded(drain_bar, 0, nullptr, kDrainLimitNs);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int e = warp - 2;                 // 0..7
+        const int lq = warp & 3;                // TMEM lane quarter this warp may access
+        const int ch = e >> 2;                  // column half: 0 -> cols 0..127, 1 -> 128..255
+        const int row_in_tile = lq * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(lq * 32) << 16;
+        int tb = 0;
+        uint32_t tphase = 0;
+        int ss = 0;
+        uint32_t sphase = 0;
+        bool ok = true;
+        float tensor_scale = 1.0f;
+        if (MODE == kModeTensor) tensor_scale = __ldg(p.sa) * __ldg(p.sb);
+
+        for (int64_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            int tm, tn, kb0, kb1, split;
+            decode_unit(p, u, tm, tn, kb0, kb1, split);
+            const int ngroups = kPromote ? (kb1 - kb0) : 1;
+            float2 acc[64];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
+
+            for (int g = 0; g < ngroups; ++g) {
+                // every lane waits; the outcome is made warp-uniform so that a
+                // lane-local timeout cannot leave a diverged warp at tcgen05.ld
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(tm_full(tb), tphase, abort_flag, kWaitLimitNs));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t sc_addr = 0;
+                float rowf = tensor_scale;
+                if (kScaleRing) {
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(sc_full(ss), sphase, abort_flag, kWaitLimitNs));
+                    if (!ok) break;
+                    const float* sc = reinterpret_cast<const float*>(smem + SmemLayout::sc_off + ss * kScaleEntryBytes);
+                    sc_addr = sbase + SmemLayout::sc_off + ss * kScaleEntryBytes;
+                    rowf = sc[row_in_tile];
+                    if (MODE == kModeBlock128) {
+                        const int off = ((tn * kBN) / 128) & 3;
+                        rowf *= sc[kBM + off + ch];
+                    }
+                }
+                const float2 rowf2 = make_float2(rowf, rowf);
+                const uint32_t tcol = tmem_base + lane_addr + (uint32_t)(tb * kBN + ch * 128);
+                // 8 chunks of 16 columns; the TMEM load of chunk c+1 is in flight
+                // while chunk c is promoted.
+                uint32_t rbuf[2][16];
+                tmem_ld_32x32b_x16(tcol, rbuf[0]);
+                tmem_ld_wait(rbuf[0]);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t (&r)[16] = rbuf[c & 1];
+                    if (c + 1 < 8) tmem_ld_32x32b_x16(tcol + (c + 1) * 16, rbuf[(c + 1) & 1]);
+                    if (kColScales) {
+                        const uint32_t sb_addr = sc_addr + (uint32_t)((kBM + ch * 128 + c * 16) * 4);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float4 b4 = lds128(sb_addr + 16 * j);
+                            const float2 f0 = fmul2(rowf2, make_float2(b4.x, b4.y));
+                            const float2 f1 = fmul2(rowf2, make_float2(b4.z, b4.w));
+                            acc[c * 8 + 2 * j] = ffma2(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), f0, acc[c * 8 + 2 * j]);
+                            acc[c * 8 + 2 * j + 1] = ffma2(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), f1, acc[c * 8 + 2 * j + 1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            acc[c * 8 + j] = ffma2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), rowf2, acc[c * 8 + j]);
+                        }
+                    }
+                    if (c + 1 < 8) tmem_ld_wait(rbuf[(c + 1) & 1]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(tm_empty(tb));
+                    if (kScaleRing) mbar_arrive(sc_empty(ss));
+                }
+                if (++tb == 2) { tb = 0; tphase ^= 1u; }
+                if (kScaleRing) {
+                    if (++ss == kScaleStages) { ss = 0; sphase ^= 1u; }
+                }
+            }
+            if (!ok) break;
+
+            // ---- store the tile: row m, columns n .. n+127 of this thread
+            const int64_t m = (int64_t)tm * kBM + row_in_tile;
+            const int n_base = tn * kBN + ch * 128;
+            if (m < p.M) {
+                if (p.splits > 1) {
+                    float* dst = p.ws + ((int64_t)split * p.M + m) * p.ldw;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = n_base + 4 * j;
+                        if (n + 4 <= p.N) {
+                            *reinterpret_cast<float4*>(dst + n) = make_float4(acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y);
+                        } else if (n < p.N) {
+                            const float v[4] = {acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y};
+                            for (int t = 0; t < p.N - n; ++t) dst[n + t] = v[t];
+                        }
+                    }
+                } else if (p.out_f32) {
+                    float* dst = reinterpret_cast<float*>(p.D) + m * p.ldd;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = n_base + 4 * j;
+                        if (n + 4 <= p.N) {
+                            *reinterpret_cast<float4*>(dst + n) = make_float4(acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y);
+                        } else if (n < p.N) {
+                            const float v[4] = {acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y};
+                            for (int t = 0; t < p.N - n; ++t) dst[n + t] = v[t];
+                        }
+                    }
+                } else {
+                    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + m * p.ldd;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int n = n_base + 8 * j;
+                        const uint4 w = make_uint4(cvt_bf16x2(acc[4 * j].x, acc[4 * j].y),
+                                                   cvt_bf16x2(acc[4 * j + 1].x, acc[4 * j + 1].y),
+                                                   cvt_bf16x2(acc[4 * j + 2].x, acc[4 * j + 2].y),
+                                                   cvt_bf16x2(acc[4 * j + 3].x, acc[4 * j + 3].y));
+                        if (n + 8 <= p.N) {
+                            *reinterpret_cast<uint4*>(dst + n) = w;
+                        } else if (n < p.N) {
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                            uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
+                            for (int t = 0; t < p.N - n; ++t)
+                                d16[n + t] = (uint16_t)((ww[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+                        }
+                    }
+                }
+            }
+        }
+        if (!ok) give_up();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// Split-K reduction: D[m,n] = sum over splits (fixed order) of ws[s][m][n].
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ ws, int splits, int64_t M,
+                                                            int64_t N, int64_t ldw, void* __restrict__ D,
+                                                            int64_t ldd, int out_f32)
+{
+    const int64_t nq = (N + 3) >> 2;          // 4-column chunks per row
+    const int64_t total = M * nq;
+    const int64_t plane = M * ldw;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = i / nq;
+        const int64_t n = (i - m * nq) << 2;
+        const float* src = ws + m * ldw + n;
+        float4 s = *reinterpret_cast<const float4*>(src);
+        for (int k = 1; k < splits; ++k) {
+            const float4 v = *reinterpret_cast<const float4*>(src + k * plane);
+            s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        }
+        const float v[4] = {s.x, s.y, s.z, s.w};
+        if (out_f32) {
+            float* d = reinterpret_cast<float*>(D) + m * ldd + n;
+            if (n + 4 <= N) *reinterpret_cast<float4*>(d) = s;
+            else for (int t = 0; t < N - n; ++t) d[t] = v[t];
+        } else {
+            __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(D) + m * ldd + n;
+            const uint32_t lo = cvt_bf16x2(s.x, s.y), hi = cvt_bf16x2(s.z, s.w);
+            if (n + 4 <= N) {
+                *reinterpret_cast<uint2*>(d) = make_uint2(lo, hi);
+            } else {
+                const uint32_t ww[2] = {lo, hi};
+                uint16_t* d16 = reinterpret_cast<uint16_t*>(d);
+                for (int t = 0; t < N - n; ++t) d16[t] = (uint16_t)((ww[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+            }
+        }
+    }
+}
+
+}  // namespace fp8bs

@@ -1,0 +1,84 @@
+"""FP8 blockwise linear forward + backward step, composed from the library's
+quantization and scaled-GEMM calls (no autograd; buffers preallocated).
+
+The composition is the one pytorch/ao PR #2785 "integrate torch._scaled_mm
+into Float8BlockwiseLinear and add bench script" benchmarks (Benchmarks table:
+eager linear forward + backward at Llama4 shapes), with the scale recipes of
+pytorch/ao PR #4209 (Findings So Far and review thread):
+
+  forward  y  = x . W^T     A = x  (1x128 along K),         B^T = W   (128x128)
+  dgrad    dx = dy . W      A = dy (1x128 along N),         B^T = W^T (128x128, same tiles)
+  wgrad    dW = dy^T . x    A = dy^T (1x128 along tokens),  B^T = x^T (1x128 along tokens)
+
+x: M x K, W: N x K, dy: M x N (all bf16); outputs bf16.  Five quantization
+launches (x, x^T, W with W^T, dy, dy^T) and three GEMM launches per step.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import ops
+
+
+class Fp8LinearStep:
+    """Preallocated buffers for one (M, N, K) linear layer's fwd + bwd."""
+
+    LAUNCHES_PER_STEP = 8
+
+    def __init__(self, M: int, N: int, K: int, device="cuda"):
+        self.M, self.N, self.K = M, N, K
+        d = device
+        u8 = torch.uint8
+        g = ops.colmajor_grid
+        cd = lambda a: (a + 127) // 128
+        # forward / dgrad operands
+        self.xq, self.xs = torch.empty((M, K), dtype=u8, device=d), g(M, cd(K), d)
+        self.wq, self.ws = torch.empty((N, K), dtype=u8, device=d), g(cd(N), cd(K), d)
+        self.wtq, self.wts = torch.empty((K, N), dtype=u8, device=d), g(cd(K), cd(N), d)
+        self.dyq, self.dys = torch.empty((M, N), dtype=u8, device=d), g(M, cd(N), d)
+        # wgrad operands (quantized along tokens, stored transposed)
+        self.dytq, self.dyts = torch.empty((N, M), dtype=u8, device=d), g(N, cd(M), d)
+        self.xtq, self.xts = torch.empty((K, M), dtype=u8, device=d), g(K, cd(M), d)
+        # outputs
+        bf = torch.bfloat16
+        self.y = torch.empty((M, N), dtype=bf, device=d)
+        self.dx = torch.empty((M, K), dtype=bf, device=d)
+        self.dW = torch.empty((N, K), dtype=bf, device=d)
+        ws = max(ops.fp8_scaled_gemm_workspace_size(M, N, K, ops.SCALE_BLOCK_1x128_128x128),
+                 ops.fp8_scaled_gemm_workspace_size(M, K, N, ops.SCALE_BLOCK_1x128_128x128),
+                 ops.fp8_scaled_gemm_workspace_size(N, K, M, ops.SCALE_BLOCK_1x128_1x128))
+        self.workspace = torch.empty((max(ws, 16),), dtype=u8, device=d)
+
+    def quantize(self, x: torch.Tensor, W: torch.Tensor, dy: torch.Tensor):
+        ops.fp8_quant_1x128(x, q=self.xq, scale_inv=self.xs)
+        ops.fp8_quant_1x128(x, transpose_out=True, q=self.xtq, scale_inv=self.xts)
+        ops.fp8_quant_128x128(W, want_q=True, want_qt=True, out=(self.wq, self.ws, self.wtq, self.wts))
+        ops.fp8_quant_1x128(dy, q=self.dyq, scale_inv=self.dys)
+        ops.fp8_quant_1x128(dy, transpose_out=True, q=self.dytq, scale_inv=self.dyts)
+
+    def gemms(self):
+        B2, B3 = ops.SCALE_BLOCK_1x128_128x128, ops.SCALE_BLOCK_1x128_1x128
+        ops.fp8_scaled_gemm(self.xq, self.wq, self.xs, self.ws, B2, out=self.y, workspace=self.workspace)
+        ops.fp8_scaled_gemm(self.dyq, self.wtq, self.dys, self.wts, B2, out=self.dx, workspace=self.workspace)
+        ops.fp8_scaled_gemm(self.dytq, self.xtq, self.dyts, self.xts, B3, out=self.dW, workspace=self.workspace)
+
+    def run(self, x: torch.Tensor, W: torch.Tensor, dy: torch.Tensor):
+        self.quantize(x, W, dy)
+        self.gemms()
+        return self.y, self.dx, self.dW
+
+    def flops(self) -> float:
+        return 3 * 2.0 * self.M * self.N * self.K
+
+    def quant_bytes(self) -> float:
+        """Algorithmic HBM bytes of the five quantization launches: bf16 read +
+        e4m3 write per element, plus 4 bytes per scale written."""
+        M, N, K = self.M, self.N, self.K
+        cd = lambda a: (a + 127) // 128
+        b = 0.0
+        b += M * K * 3 + 4 * M * cd(K)            # x 1x128
+        b += M * K * 3 + 4 * K * cd(M)            # x^T along tokens
+        b += N * K * 4 + 2 * 4 * cd(N) * cd(K)    # W 128x128 + transposed copy (2 B in, 2 x 1 B out)
+        b += M * N * 3 + 4 * M * cd(N)            # dy 1x128
+        b += M * N * 3 + 4 * N * cd(M)            # dy^T along tokens
+        return b

@@ -1,0 +1,228 @@
+"""Python binding of libfp8bs (the C ABI in include/fp8bs.h).
+
+Argument marshalling only: every function here checks the tensors' device,
+allocates outputs with torch when they are not given, and calls the C entry
+point of the same name with raw pointers and torch's current CUDA stream.  All
+arithmetic happens in the CUDA library; if the library is missing or was not
+built, the first call raises -- there is no fallback path.
+
+Scale grids are column-major fp32, as the library writes and reads them.  In
+torch they are returned as (rows, groups) views with strides (1, ld): element
+[i, j] is the scale of row i, group j, stored at i + j*ld.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+FP8BS_OK = 0
+STATUS_NAMES = {
+    0: "FP8BS_OK", 1: "FP8BS_ERR_INVALID_ARG", 2: "FP8BS_ERR_UNSUPPORTED", 3: "FP8BS_ERR_ALIGNMENT",
+    4: "FP8BS_ERR_WORKSPACE", 5: "FP8BS_ERR_CUDA", 6: "FP8BS_ERR_TIMEOUT", 7: "FP8BS_ERR_NO_SM100",
+}
+
+BF16, F32 = 0, 1
+SCALE_TENSOR, SCALE_ROWWISE, SCALE_BLOCK_1x128_128x128, SCALE_BLOCK_1x128_1x128 = 0, 1, 2, 3
+SCALE_COL_MAJOR = 0
+
+_lib = None
+
+
+class Fp8bsError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+def lib():
+    """Load libfp8bs.so (built in-tree).  Raises if it is absent."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB_PATH
+        if not os.path.exists(path):
+            raise ImportError(f"libfp8bs.so not built ({path}); run fp8_block_scaled_11_b200/build.py")
+        L = ctypes.CDLL(path)
+        p, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.fp8_quant_1x128.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, i32, p]
+        L.fp8_quant_128x128.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, p, i64, p, i64, p]
+        L.fp8_quant_tensor_workspace_size.argtypes = [i64]
+        L.fp8_quant_tensor_workspace_size.restype = sz
+        L.fp8_quant_tensor.argtypes = [p, i32, i64, p, p, p, sz, p]
+        L.fp8_quant_rowwise.argtypes = [p, i32, i64, i64, i64, p, i64, p, p]
+        L.fp8_scaled_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
+        L.fp8_scaled_gemm_workspace_size.restype = sz
+        L.fp8_scaled_gemm.argtypes = [i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, i32, p, i64, i32, p, sz, p]
+        L.fp8bs_status_string.argtypes = [i32]
+        L.fp8bs_status_string.restype = ctypes.c_char_p
+        L.fp8bs_check_device_error.argtypes = [p]
+        for fn in ("fp8_quant_1x128", "fp8_quant_128x128", "fp8_quant_tensor", "fp8_quant_rowwise",
+                   "fp8_scaled_gemm", "fp8bs_check_device_error"):
+            getattr(L, fn).restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != FP8BS_OK:
+        raise Fp8bsError(fn, status)
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported input dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ld(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D row-major tensor (unit column stride)")
+    return t.stride(0)
+
+
+def _round_up(x: int, m: int) -> int:
+    return (x + m - 1) // m * m
+
+
+def colmajor_grid(rows: int, groups: int, device) -> torch.Tensor:
+    """Allocate a column-major fp32 scale grid (rows x groups), ld = rows rounded up to 4."""
+    ld = _round_up(max(rows, 1), 4)
+    return torch.empty((groups, ld), dtype=torch.float32, device=device)[:, :rows].t()
+
+
+def _grid_ld(s: torch.Tensor, rows: int) -> int:
+    if s.dim() != 2 or s.dtype != torch.float32:
+        raise ValueError("scale grid must be a 2-D fp32 tensor")
+    if s.shape[1] == 1:
+        return s.stride(1) if s.stride(0) == 1 and s.stride(1) >= rows else _round_up(rows, 4)
+    if s.stride(0) != 1:
+        raise ValueError("scale grid must be column-major (stride (1, ld))")
+    return s.stride(1)
+
+
+# ---------------------------------------------------------------------------- quantization
+def fp8_quant_1x128(x: torch.Tensor, transpose_out: bool = False, q: Optional[torch.Tensor] = None,
+                    scale_inv: Optional[torch.Tensor] = None):
+    """Returns (q uint8, scale_inv grid).  transpose_out=False: q is rows x cols,
+    grid rows x ceil(cols/128).  transpose_out=True: groups run along rows and
+    q is the quantized transpose (cols x rows), grid cols x ceil(rows/128).
+    Preallocated outputs may be passed as q / scale_inv."""
+    rows, cols = x.shape
+    xt = _dtype_code(x)
+    out_rows, out_cols = (cols, rows) if transpose_out else (rows, cols)
+    if q is None:
+        q = torch.empty((out_rows, out_cols), dtype=torch.uint8, device=x.device)
+    s = scale_inv if scale_inv is not None else colmajor_grid(out_rows, (out_cols + 127) // 128, x.device)
+    ld_s = _grid_ld(s, out_rows)
+    _check("fp8_quant_1x128", lib().fp8_quant_1x128(x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(), q.stride(0),
+                                                    s.data_ptr(), ld_s, int(transpose_out), _stream(x)))
+    return q, s
+
+
+def fp8_quant_128x128(x: torch.Tensor, want_q: bool = True, want_qt: bool = False, out=None):
+    """Returns (q, scale_inv, q_t, scale_inv_t); the unrequested pair is None.
+    q: rows x cols, grid ceil(rows/128) x ceil(cols/128).  q_t: cols x rows
+    (the same quantized tiles transposed), grid ceil(cols/128) x ceil(rows/128).
+    Preallocated outputs may be passed as out=(q, s, q_t, s_t)."""
+    rows, cols = x.shape
+    xt = _dtype_code(x)
+    rb, cb = (rows + 127) // 128, (cols + 127) // 128
+    q = s = qt = st = None
+    if out is not None:
+        q, s, qt, st = out
+    qp = sp = qtp = stp = 0
+    ldq = lds = ldqt = ldst = 0
+    if want_q:
+        if q is None:
+            q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+            s = colmajor_grid(rb, cb, x.device)
+        qp, sp, ldq, lds = q.data_ptr(), s.data_ptr(), q.stride(0), _grid_ld(s, rb)
+    if want_qt:
+        if qt is None:
+            qt = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+            st = colmajor_grid(cb, rb, x.device)
+        qtp, stp, ldqt, ldst = qt.data_ptr(), st.data_ptr(), qt.stride(0), _grid_ld(st, cb)
+    _check("fp8_quant_128x128", lib().fp8_quant_128x128(x.data_ptr(), xt, rows, cols, _ld(x), qp, ldq, sp, lds,
+                                                        qtp, ldqt, stp, ldst, _stream(x)))
+    return q, s, qt, st
+
+
+def fp8_quant_tensor(x: torch.Tensor, workspace: Optional[torch.Tensor] = None):
+    """Returns (q, scale_inv[1])."""
+    n = x.numel()
+    xc = x.contiguous()
+    xt = _dtype_code(x)
+    q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    s = torch.empty((1,), dtype=torch.float32, device=x.device)
+    wsb = lib().fp8_quant_tensor_workspace_size(n)
+    if workspace is None:
+        workspace = torch.empty((wsb,), dtype=torch.uint8, device=x.device)
+    _check("fp8_quant_tensor", lib().fp8_quant_tensor(xc.data_ptr(), xt, n, q.data_ptr(), s.data_ptr(),
+                                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                                      _stream(x)))
+    return q, s
+
+
+def fp8_quant_rowwise(x: torch.Tensor):
+    """Returns (q, scale_inv[rows])."""
+    rows, cols = x.shape
+    xt = _dtype_code(x)
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    s = torch.empty((rows,), dtype=torch.float32, device=x.device)
+    _check("fp8_quant_rowwise", lib().fp8_quant_rowwise(x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(),
+                                                        q.stride(0), s.data_ptr(), _stream(x)))
+    return q, s
+
+
+# ---------------------------------------------------------------------------- GEMM
+def fp8_scaled_gemm_workspace_size(M: int, N: int, K: int, mode: int) -> int:
+    return int(lib().fp8_scaled_gemm_workspace_size(M, N, K, mode))
+
+
+def fp8_scaled_gemm(A: torch.Tensor, Bt: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor, mode: int,
+                    out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, split_k: bool = True) -> torch.Tensor:
+    """D = scaled(A . Bt^T).  A: M x K uint8 (e4m3), Bt: N x K uint8 (e4m3).
+    Scales as returned by the quantization functions (TENSOR: 1 element;
+    ROWWISE: M / N elements; BLOCK: column-major grids)."""
+    M, K = A.shape
+    N, K2 = Bt.shape
+    if K2 != K:
+        raise ValueError("A and Bt must share K")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    oc = F32 if out.dtype == torch.float32 else BF16
+    if mode in (SCALE_BLOCK_1x128_128x128, SCALE_BLOCK_1x128_1x128):
+        ld_sa = _grid_ld(scale_a, M)
+        ld_sb = _grid_ld(scale_b, scale_b.shape[0])
+    else:
+        ld_sa = ld_sb = 0
+    wsb = fp8_scaled_gemm_workspace_size(M, N, K, mode) if split_k else 0
+    if wsb > 0 and workspace is None:
+        workspace = torch.empty((wsb,), dtype=torch.uint8, device=A.device)
+    wp = workspace.data_ptr() if (workspace is not None and wsb > 0) else 0
+    wn = workspace.numel() * workspace.element_size() if (workspace is not None and wsb > 0) else 0
+    _check("fp8_scaled_gemm", lib().fp8_scaled_gemm(M, N, K, A.data_ptr(), _ld(A), Bt.data_ptr(), _ld(Bt),
+                                                    scale_a.data_ptr(), ld_sa, scale_b.data_ptr(), ld_sb, mode,
+                                                    SCALE_COL_MAJOR, out.data_ptr(), _ld(out), oc, wp, wn,
+                                                    _stream(A)))
+    return out
+
+
+def fp8bs_status_string(status: int) -> str:
+    return lib().fp8bs_status_string(status).decode()
+
+
+def fp8bs_check_device_error(stream: Optional[torch.cuda.Stream] = None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(lib().fp8bs_check_device_error(ctypes.c_void_p(s.cuda_stream)))

@@ -1,0 +1,214 @@
+/*
+ * fp8bs.h -- C ABI of libfp8bs: FP8 (e4m3) dynamic quantization and scaled
+ * GEMM for NVIDIA B200 (sm_100a).
+ *
+ * The operations (see each function for the passage that defines it):
+ *
+ *   quantize     a group G of inputs (1x128 slice, 128x128 tile, row, tensor):
+ *                amax = max|x| over G, s = 448 / max(amax, 1e-12) in fp32
+ *                (IEEE), q = e4m3(x * s) rounded to nearest even and saturated
+ *                to +-448, and the reciprocal r = 1/s is stored as the scale.
+ *   scaled GEMM  C[m,n] = sum_kb  rA(m,kb) * rB(n,kb) * sum_{k in block kb} qA[m,k] qB[n,k]
+ *                with K blocks of 128, fp32 accumulation on the tensor cores,
+ *                per-K-block promotion of the partial sums in fp32 registers,
+ *                bf16 or fp32 output.
+ *
+ * e4m3 is the OCP 8-bit E4M3 format (bias 7, no infinities, max 448).
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory and keeps no device state except one int of
+ *     device-side error flag (see fp8bs_check_device_error).
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream) and
+ *     never synchronizes, except fp8bs_check_device_error.
+ *   - Arguments are validated before anything is launched; on an error status
+ *     nothing has been launched and no output was touched.
+ *   - Matrices are row-major with an explicit leading dimension in ELEMENTS.
+ *     Scale grids are column-major fp32 with an explicit leading dimension:
+ *     the scale of (row i, block j) lives at scale[i + j*ld].
+ *   - Inputs must be finite (NaN/Inf inputs are outside the contract).
+ *   - Only compute capability 10.x devices (B200, sm_100a) are supported;
+ *     anything else returns FP8BS_ERR_NO_SM100.  There is no fallback path.
+ */
+#ifndef FP8BS_H
+#define FP8BS_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8BS_OK = 0,
+    FP8BS_ERR_INVALID_ARG = 1,   /* null pointer, size < 1, ld too small, bad flag      */
+    FP8BS_ERR_UNSUPPORTED = 2,   /* unknown enum value                                  */
+    FP8BS_ERR_ALIGNMENT = 3,     /* pointer / leading dimension / size alignment rule   */
+    FP8BS_ERR_WORKSPACE = 4,     /* workspace given but smaller than required           */
+    FP8BS_ERR_CUDA = 5,          /* a CUDA runtime/driver call or launch failed         */
+    FP8BS_ERR_TIMEOUT = 6,       /* a device-side wait ran past its limit (see below)   */
+    FP8BS_ERR_NO_SM100 = 7       /* current device is not compute capability 10.x     */
+} fp8bs_status;
+
+typedef enum { FP8BS_BF16 = 0, FP8BS_F32 = 1 } fp8bs_dtype;
+
+typedef enum {
+    FP8BS_SCALE_TENSOR = 0,              /* rA = scale_a[0],              rB = scale_b[0]               */
+    FP8BS_SCALE_ROWWISE = 1,             /* rA = scale_a[m],              rB = scale_b[n]               */
+    FP8BS_SCALE_BLOCK_1x128_128x128 = 2, /* rA = scale_a[m + kb*ld_sa],   rB = scale_b[n/128 + kb*ld_sb] */
+    FP8BS_SCALE_BLOCK_1x128_1x128 = 3    /* rA = scale_a[m + kb*ld_sa],   rB = scale_b[n + kb*ld_sb]     */
+} fp8bs_scale_mode;
+
+typedef enum { FP8BS_SCALE_COL_MAJOR = 0 } fp8bs_scale_layout;
+
+/*
+ * fp8_quant_1x128 -- dynamic quantization with one scale per 1x128 group.
+ *
+ * Defined by: pytorch/ao PR #2592 "add more generic kernel for fp8 blockwise
+ * scaling" (Performance table, block shape (1,128)); pytorch/ao PR #2785
+ * "integrate torch._scaled_mm into Float8BlockwiseLinear and add bench
+ * script" (Summary: column-major scales, reciprocal scales written directly
+ * by the quant kernel).
+ *
+ * x          rows x cols, dtype xt (bf16 or fp32), leading dim ldx elements.
+ * transpose_out = 0: groups run along the contiguous dim (cols).
+ *            q:          rows x cols e4m3 bytes, leading dim ldq.
+ *            scale_inv:  grid rows x ceil(cols/128), scale_inv[r + g*ld_scale],
+ *                        ld_scale >= rows.
+ * transpose_out = 1: groups run along the rows of x ("scaled along tokens"),
+ *            and the quantized TRANSPOSE is written:
+ *            q:          cols x rows e4m3 bytes, q[c*ldq + r], leading dim ldq >= rows.
+ *            scale_inv:  grid cols x ceil(rows/128), scale_inv[c + g*ld_scale],
+ *                        ld_scale >= cols.
+ * A ragged last group (size not a multiple of 128) is quantized over its valid
+ * elements only.
+ * Alignment: x, q, scale_inv 16-byte aligned; ldx*sizeof(xt) and ldq multiples
+ * of 16 bytes; cols % 16 == 0 (and rows % 16 == 0 when transpose_out);
+ * ld_scale % 4 == 0.  Otherwise FP8BS_ERR_ALIGNMENT.
+ */
+fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                             uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale,
+                             int transpose_out, cudaStream_t stream);
+
+/*
+ * fp8_quant_128x128 -- dynamic quantization with one scale per 128x128 tile.
+ *
+ * Defined by: pytorch/ao PR #2592 (Performance table, block shape (128,128));
+ * the weight side of the (BlockWise1x128, BlockWise128x128) recipe in
+ * pytorch/ao PR #4209 "[codex] add repro for blockwise _scaled_mm
+ * investigation" (Findings So Far); 2-D tile loads as in PR #2785's stack
+ * ("load 2d chunks for groupwise quant to enable coalesced gmem accesses").
+ *
+ * x            rows x cols, dtype xt, leading dim ldx.
+ * q            (nullable) rows x cols e4m3, leading dim ldq.
+ * scale_inv    grid ceil(rows/128) x ceil(cols/128), scale_inv[bi + bj*ld_scale],
+ *              ld_scale >= ceil(rows/128).  Required when q != NULL.
+ * q_t          (nullable) the same quantized tile bytes transposed: cols x rows,
+ *              q_t[c*ldq_t + r], leading dim ldq_t >= rows.
+ * scale_inv_t  the transposed grid ceil(cols/128) x ceil(rows/128),
+ *              scale_inv_t[bj + bi*ld_scale_t], ld_scale_t >= ceil(cols/128).
+ *              Required when q_t != NULL.
+ * At least one of q, q_t must be non-NULL.  Edge tiles are quantized over
+ * their valid elements only.
+ * Alignment: pointers 16-byte aligned; ldx*sizeof(xt), ldq, ldq_t multiples of
+ * 16 bytes; rows % 16 == 0 and cols % 16 == 0; ld_scale, ld_scale_t % 4 == 0.
+ */
+fp8bs_status fp8_quant_128x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                               uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale,
+                               uint8_t* q_t, int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t,
+                               cudaStream_t stream);
+
+/*
+ * fp8_quant_tensor -- dynamic quantization with one scale for the whole tensor.
+ *
+ * Defined by: ROCm/aiter issue #1765 "[Issue]: Does gemm_a8w8 support
+ * per-tensor quant?" (Steps to Reproduce: per_tensor_quant returns the
+ * quantized tensor and a single dequantization scale, dequant = q * scale).
+ *
+ * x          n contiguous elements of dtype xt.
+ * q          n e4m3 bytes.
+ * scale_inv  one float (the dequantization scale 1/s).
+ * workspace  device scratch of at least fp8_quant_tensor_workspace_size(n)
+ *            bytes, 16-byte aligned; no initial contents needed.  Two launches
+ *            (amax partials, then quantize) share it on `stream`.
+ * Alignment: x, q 16-byte aligned; n % 16 == 0.
+ */
+size_t fp8_quant_tensor_workspace_size(int64_t n);
+fp8bs_status fp8_quant_tensor(const void* x, fp8bs_dtype xt, int64_t n, uint8_t* q, float* scale_inv,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fp8_quant_rowwise -- dynamic quantization with one scale per row.
+ *
+ * Defined by: the rowwise variant of scaled_mm (pytorch/pytorch issue #159940,
+ * Describe the bug: the scaled_mm template's SCALING_ROWWISE flag); applied to
+ * x (per row) and to W (per row of W = per output column).
+ *
+ * x          rows x cols, dtype xt, leading dim ldx.
+ * q          rows x cols e4m3, leading dim ldq.
+ * scale_inv  rows floats.
+ * Alignment: x, q 16-byte aligned; ldx*sizeof(xt), ldq multiples of 16 bytes;
+ * cols % 16 == 0; scale_inv 4-byte aligned.
+ */
+fp8bs_status fp8_quant_rowwise(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                               uint8_t* q, int64_t ldq, float* scale_inv, cudaStream_t stream);
+
+/*
+ * fp8_scaled_gemm -- D = scaled (A . Bt^T), the "TN" layout of F.linear.
+ *
+ * Defined by: the explicit dequantized matmul of pytorch/ao PR #4209 (What
+ * Changed: FP32 reference, dequantized matmul and kernels on the same
+ * quantized inputs and reciprocal scales) and of ROCm/aiter issue #1765 (Steps
+ * to Reproduce: F.linear(q_x*s_x, q_w*s_w)); recipes (1x128, 128x128) and
+ * (1x128, 1x128) from PR #4209 (Findings So Far and its review thread),
+ * per-tensor from issue #1765, rowwise from pytorch/pytorch issue #159940.
+ *
+ * A          M x K e4m3, leading dim lda (bytes).
+ * Bt         N x K e4m3, leading dim ldb (bytes): row n holds column n of B.
+ * scale_a    TENSOR: 1 float.  ROWWISE: M floats.  BLOCK_*: grid M x ceil(K/128),
+ *            scale_a[m + kb*ld_sa], ld_sa >= M.
+ * scale_b    TENSOR: 1 float.  ROWWISE: N floats.
+ *            BLOCK_1x128_128x128: grid ceil(N/128) x ceil(K/128), scale_b[nb + kb*ld_sb],
+ *            ld_sb >= ceil(N/128) (as written by fp8_quant_128x128 on Bt).
+ *            BLOCK_1x128_1x128: grid N x ceil(K/128), scale_b[n + kb*ld_sb], ld_sb >= N.
+ * D          M x N, dtype out_dtype (bf16 rounded to nearest even, or fp32),
+ *            leading dim ldd elements.
+ * workspace  optional fp32 scratch for split-K (used when the output has too few
+ *            128x256 tiles to fill the GPU).  Pass NULL/0 to disable split-K, or
+ *            at least fp8_scaled_gemm_workspace_size(M, N, K, mode) bytes.  The
+ *            split partial sums are added in a fixed order: results are
+ *            deterministic.
+ * Any M, N >= 1 and any K >= 16 with K % 16 == 0 (any number of K blocks;
+ * a ragged last K block contributes its valid columns only).
+ * Alignment: A, Bt, D, scale_a, scale_b, workspace 16-byte aligned; lda, ldb
+ * multiples of 16; ldd*sizeof(out) a multiple of 16; ld_sa, ld_sb % 4 == 0 for
+ * the block modes.
+ */
+size_t fp8_scaled_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8bs_scale_mode mode);
+fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K,
+                             const uint8_t* A, int64_t lda, const uint8_t* Bt, int64_t ldb,
+                             const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
+                             fp8bs_scale_mode mode, fp8bs_scale_layout layout,
+                             void* D, int64_t ldd, fp8bs_dtype out_dtype,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* fp8bs_status_string(fp8bs_status s);
+
+/*
+ * fp8bs_check_device_error -- synchronizes `stream`, then reads and clears the
+ * library's device-side error flag.  The GEMM kernel bounds every wait on its
+ * internal pipeline barriers (a few seconds); a wait that runs out sets the
+ * flag, the kernel drains its copies in flight, frees its tensor memory and
+ * returns, so the CUDA context stays usable.  Returns FP8BS_ERR_TIMEOUT if the
+ * flag was set, FP8BS_ERR_CUDA if the stream reports an error, else FP8BS_OK.
+ */
+fp8bs_status fp8bs_check_device_error(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BS_H */
