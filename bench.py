@@ -1,0 +1,412 @@
+"""Benchmark of the FP8 blockwise hot path on B200.
+
+One step = the Llama4-shape FP8 linear forward + backward for both layer
+shapes (N, K) = (5120, 8192) and (8192, 5120) at M = 16640 tokens: per shape
+five dynamic-quantization launches (x 1x128, x^T along tokens, W 128x128 with
+its transpose, dy 1x128, dy^T along tokens) and three scaled GEMMs (forward
+and dgrad with 1x128 x 128x128 scales, wgrad with 1x128 x 1x128), bf16 out.
+This is the workload of pytorch/ao PR #2785 "integrate torch._scaled_mm into
+Float8BlockwiseLinear and add bench script" (Benchmarks table).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs the same per-GPU
+workload on its own batch (weak scaling, no collective on the data path); the
+time is the max over ranks.  `--impl reference` times the CPU oracle instead
+(rank 0 only), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "blockwise FP8 GEMM TFLOP/s (% of B200 FP8 peak); quant GB/s (% of HBM)"
+UNIT = "TFLOP/s"
+# The pages' own figure for this workload: fp8 torch._scaled_mm eager fwd+bwd,
+# 7746.98 us at (5120, 8192) and 7783.31 us at (8192, 5120), hardware not stated.
+PAGES_FP8_US = (7746.98, 7783.31)
+FP8_SPEC_TFLOPS = 4500.0
+
+# DRAM traffic of one GEMM launch from an ncu capture, keyed by the SHA-256 of
+# the kernel source it was taken on (profiles/ holds the summary).  A changed
+# kernel reports null until it is captured again.
+GEMM_TRAFFIC = {}
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for f in ("gemm_kernel.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "fp8_block_scaled_11_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        mhz, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------------ GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from fp8_block_scaled_11_b200 import inputs, ops
+    from fp8_block_scaled_11_b200.linear import Fp8LinearStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    ops.lib()
+    M = inputs.LLAMA4_M
+    shapes = inputs.LLAMA4_SHAPES
+    steps = [Fp8LinearStep(M, N, K) for N, K in shapes]
+    data = []
+    for N, K in shapes:
+        x, W, dy = inputs.llama4(N, K)
+        data.append((x, W, dy))
+    dev_data = [tuple(t.cuda() for t in d) for d in data]
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def one_step(events=None):
+        for st, (x, W, dy) in zip(steps, dev_data):
+            if events is None:
+                st.run(x, W, dy)
+            else:
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                e[0].record(stream)
+                st.quantize(x, W, dy)
+                e[1].record(stream)
+                st.gemms()
+                e[2].record(stream)
+                events.append((st, e))
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    st_err = ops.fp8bs_check_device_error()
+    if st_err != 0:
+        raise SystemExit(f"device error after warm-up: {ops.fp8bs_status_string(st_err)}")
+
+    # ---- timed region: K steps, CUDA events on the launching stream
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    events = []
+    t0.record(stream)
+    for _ in range(args.steps):
+        one_step(events)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms_total = t0.elapsed_time(t1)
+    quant_ms = sum(e[0].elapsed_time(e[1]) for _, e in events)
+    gemm_ms = sum(e[1].elapsed_time(e[2]) for _, e in events)
+    if world > 1:
+        tt = torch.tensor([ms_total, quant_ms, gemm_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total, quant_ms, gemm_ms = tt.tolist()
+
+    flops_step = sum(st.flops() for st in steps)
+    qbytes_step = sum(st.quant_bytes() for st in steps)
+    ms_step = ms_total / args.steps
+    value = world * flops_step * args.steps / (ms_total * 1e-3) / 1e12
+    gemm_tflops = flops_step * args.steps / (gemm_ms * 1e-3) / 1e12
+    gemm_launches = 3 * len(steps) * args.steps
+    gemm_avg_us = gemm_ms * 1e3 / gemm_launches
+    quant_gbs = qbytes_step * args.steps / (quant_ms * 1e-3) / 1e9
+
+    peaks, peak_src = measured_peaks()
+    timed_region_s = ms_total * 1e-3
+    sustained = timed_region_s > 2.0
+    bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    fp8_peak = 2.0 * bf16          # fp8 / bf16 dense ratio 4.5 / 2.25
+    tr = GEMM_TRAFFIC.get(kernel_hash())
+
+    # ---- end to end: host (pinned) inputs -> device, the step, results -> host
+    e2e = None
+    if not args.no_e2e:
+        host_in = [tuple(t.pin_memory() for t in d) for d in data]
+        host_out = [tuple(torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in (st.y, st.dx, st.dW))
+                    for st in steps]
+        n_e2e = max(1, min(args.steps, 10))
+
+        def e2e_step():
+            for st, (xh, Wh, dyh), outs in zip(steps, host_in, host_out):
+                x = xh.to("cuda", non_blocking=True)
+                W = Wh.to("cuda", non_blocking=True)
+                dy = dyh.to("cuda", non_blocking=True)
+                y, dx, dW = st.run(x, W, dy)
+                for o, d in zip(outs, (y, dx, dW)):
+                    o.copy_(d, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            tt = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = tt.item()
+        bi = sum(sum(t.numel() * t.element_size() for t in d) for d in host_in)
+        bo = sum(sum(t.numel() * t.element_size() for t in o) for o in host_out)
+        e2e = {"value": round(world * flops_step * n_e2e / (e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": n_e2e,
+               "path": "pinned host tensors -> ops (C ABI) -> pinned host tensors"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(args.cpu_rows)
+
+    pages_tflops = 2 * 3 * 2.0 * M * 5120 * 8192 / (sum(PAGES_FP8_US) * 1e-6) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": round(value / world / pages_tflops, 3),
+        "dtype": "e4m3 x e4m3 -> fp32 accumulate, bf16 out", "data": "synthetic (seeded N(0,1) / kaiming-uniform bf16)",
+        "config": {
+            "workload": "Llama4-shape FP8 linear fwd+bwd, M=16640, (N,K)=(5120,8192) and (8192,5120); "
+                        "fwd/dgrad 1x128 x 128x128, wgrad 1x128 x 1x128 (along tokens); dynamic quant included",
+            "parallelism": f"dp{world} (independent per-GPU batches, no data-path collective)",
+            "l2": "inputs larger than L2 (x alone is 272 MB); no flush",
+            "vs_baseline_ref": f"pages' fp8 _scaled_mm eager fwd+bwd ({PAGES_FP8_US[0]}+{PAGES_FP8_US[1]} us, "
+                               f"hardware not stated) = {pages_tflops:.1f} TFLOP/s per GPU",
+        },
+        "breakdown": {
+            "gemm_tflops": round(gemm_tflops, 1),
+            "gemm_frac_of_fp8_spec": round(gemm_tflops / FP8_SPEC_TFLOPS, 3),
+            "quant_gbs": round(quant_gbs, 1),
+            "quant_frac_of_hbm": round(quant_gbs / peaks["hbm_gbs"], 3),
+            "quant_ms_per_step": round(quant_ms / args.steps, 4),
+            "gemm_ms_per_step": round(gemm_ms / args.steps, 4),
+        },
+        "roofline": {
+            "kernel": "gemm_fp8_kernel (6 launches per step)",
+            "bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+            "frac": round(gemm_tflops / fp8_peak, 3), "traffic": tr,
+            "peak_source": f"2 x {'sustained' if sustained else 'burst'} bf16 of {peak_src} "
+                           f"({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'fallback'}), fp8/bf16 ratio 2",
+            "avg_launch_us": round(gemm_avg_us, 1),
+        },
+        "clocks": clocks,
+        "gpu_launches": Fp8LinearStep.LAUNCHES_PER_STEP * len(steps) * args.steps,
+        "e2e": e2e,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------ oracle (CPU) arm
+class OracleSample:
+    """The oracle, as it stands, on a bounded sample of the same workload.  Per
+    layer shape and per step: quantize (1x128) `rows` token rows of x and dy,
+    the first 128-row band of W (128x128) and of W^T, and the first 128 rows of
+    x^T and dy^T along all tokens; then compute, in fp64, output rows x the
+    first 128 columns of the forward and dgrad GEMMs and the first 128 x 128
+    block of the wgrad GEMM.  Value = the sampled GEMM FLOPs / wall time of the
+    quantization + GEMM calls (input generation excluded)."""
+
+    def __init__(self, rows: int):
+        import numpy as np
+        import torch
+
+        import oracle
+        from fp8_block_scaled_11_b200 import inputs
+
+        oracle.lib()
+        self.oracle = oracle
+        self.rows = rows
+        self.data = []
+        for N, K in inputs.LLAMA4_SHAPES:
+            x, W, dy = inputs.llama4(N, K)
+            self.data.append((N, K, x.view(torch.uint16).numpy(), W.view(torch.uint16).numpy(),
+                              dy.view(torch.uint16).numpy()))
+        self.M = inputs.LLAMA4_M
+        self.idx = np.arange(rows, dtype=np.int64)
+        self.band = np.arange(128, dtype=np.int64)
+
+    def step(self):
+        o = self.oracle
+        flops = 0.0
+        t = time.perf_counter()
+        for N, K, xb, Wb, dyb in self.data:
+            qx, sx = o.quant_1x128(xb, rows=self.idx)
+            qw, sw = o.quant_128x128(Wb, rblocks=[0])                  # W rows 0..127
+            qwt, swt = o.quant_128x128(Wb, transpose=True, rblocks=[0])  # W^T rows 0..127
+            qdy, sdy = o.quant_1x128(dyb, rows=self.idx)
+            qdyt, sdyt = o.quant_1x128(dyb, transpose=True, rows=self.band)
+            qxt, sxt = o.quant_1x128(xb, transpose=True, rows=self.band)
+            o.gemm(qx, qw, sx, sw, o.SCALE_BLOCK_1x128_128x128)
+            o.gemm(qdy, qwt, sdy, swt, o.SCALE_BLOCK_1x128_128x128)
+            o.gemm(qdyt, qxt, sdyt, sxt, o.SCALE_BLOCK_1x128_1x128)
+            flops += 2.0 * (self.rows * 128 * K + self.rows * 128 * N + 128 * 128 * self.M)
+        secs = time.perf_counter() - t
+        return flops, secs
+
+    def describe(self):
+        return (f"per layer shape and step: {self.rows} token rows x 128 output columns of fwd and dgrad, "
+                f"a 128x128 block of wgrad over all 16640 tokens, with the quantization those need "
+                f"(W / W^T 128-row bands, x / dy rows, x^T / dy^T 128-row bands); fp64 GEMM oracle")
+
+
+def _cores():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline_sample(rows: int, budget_s: float = 12.0):
+    """Timed oracle sample for the main line (about budget_s of CPU work)."""
+    smp = OracleSample(rows)
+    flops = secs = 0.0
+    n = 0
+    while secs < budget_s and n < 50:
+        f, s_ = smp.step()
+        flops += f
+        secs += s_
+        n += 1
+    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "seconds": round(secs, 2), "sample": f"{n} sampled steps; " + smp.describe()}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    smp = OracleSample(args.cpu_rows)
+    for _ in range(args.warmup):
+        smp.step()
+    flops = secs = 0.0
+    for _ in range(args.steps):
+        f, s_ = smp.step()
+        flops += f
+        secs += s_
+    value = round(flops / secs / 1e12, 6)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs * 1e3 / args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic (seeded N(0,1) / kaiming-uniform bf16)",
+        "config": {"workload": "Llama4-shape FP8 linear fwd+bwd, M=16640, (N,K)=(5120,8192) and (8192,5120); "
+                               "each step a bounded sample (see cpu_baseline.sample)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                         "sample": smp.describe()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=32)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

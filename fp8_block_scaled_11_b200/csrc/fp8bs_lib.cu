@@ -364,9 +364,10 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
         if (mode == FP8BS_SCALE_BLOCK_1x128_1x128 && ld_sb < N) return FP8BS_ERR_INVALID_ARG;
         if (ld_sa % 4 || ld_sb % 4) return FP8BS_ERR_ALIGNMENT;
     }
-    if (K % 16 || lda % 16 || ldb % 16 || (ldd * (int64_t)dtype_size(out_dtype)) % 16) return FP8BS_ERR_ALIGNMENT;
-    if (!aligned16(A) || !aligned16(Bt) || !aligned16(D) || !aligned16(scale_a) || !aligned16(scale_b))
-        return FP8BS_ERR_ALIGNMENT;
+    if (K % 16 || lda % 16 || ldb % 16) return FP8BS_ERR_ALIGNMENT;
+    if (!aligned16(A) || !aligned16(Bt) || !aligned16(scale_a) || !aligned16(scale_b)) return FP8BS_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(D) % dtype_size(out_dtype)) return FP8BS_ERR_ALIGNMENT;
+    const int vec_out = aligned16(D) && (ldd * (int64_t)dtype_size(out_dtype)) % 16 == 0;
     DeviceInfo* d = nullptr;
     fp8bs_status st = get_device(&d);
     if (st != FP8BS_OK) return st;
@@ -420,6 +421,7 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
     p.D = D;
     p.ldd = ldd;
     p.out_f32 = out_dtype == FP8BS_F32;
+    p.vec_out = vec_out;
     p.ws = static_cast<float*>(workspace);
     p.ldw = plan.ldw;
     p.sa = scale_a;
@@ -436,7 +438,7 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
     if (plan.splits > 1) {
         const int64_t chunks = M * ((N + 3) / 4);
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(chunks, 256), (int64_t)d->num_sms * 8));
-        splitk_reduce_kernel<<<grid, 256, 0, stream>>>(p.ws, plan.splits, M, N, plan.ldw, D, ldd, p.out_f32);
+        splitk_reduce_kernel<<<grid, 256, 0, stream>>>(p.ws, plan.splits, M, N, plan.ldw, D, ldd, p.out_f32, vec_out);
         st = launch_status();
     }
     return st;

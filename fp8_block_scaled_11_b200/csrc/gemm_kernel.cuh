@@ -80,6 +80,7 @@ struct GemmParams {
     void* D;                    // output (bf16 or fp32) when splits == 1
     int64_t ldd;
     int32_t out_f32;
+    int32_t vec_out;            // 1: D and ldd allow 16-byte row-chunk stores
     float* ws;                  // split-K partials [splits][M][ldw] fp32
     int64_t ldw;
     const float* sa;            // tensor mode: scale pointers read directly
@@ -370,11 +371,11 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int n = n_base + 4 * j;
-                        if (n + 4 <= p.N) {
+                        if (p.vec_out && n + 4 <= p.N) {
                             *reinterpret_cast<float4*>(dst + n) = make_float4(acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y);
                         } else if (n < p.N) {
                             const float v[4] = {acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y};
-                            for (int t = 0; t < p.N - n; ++t) dst[n + t] = v[t];
+                            for (int t = 0; t < min(4, p.N - n); ++t) dst[n + t] = v[t];
                         }
                     }
                 } else {
@@ -386,12 +387,12 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                                                    cvt_bf16x2(acc[4 * j + 1].x, acc[4 * j + 1].y),
                                                    cvt_bf16x2(acc[4 * j + 2].x, acc[4 * j + 2].y),
                                                    cvt_bf16x2(acc[4 * j + 3].x, acc[4 * j + 3].y));
-                        if (n + 8 <= p.N) {
+                        if (p.vec_out && n + 8 <= p.N) {
                             *reinterpret_cast<uint4*>(dst + n) = w;
                         } else if (n < p.N) {
                             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
                             uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
-                            for (int t = 0; t < p.N - n; ++t)
+                            for (int t = 0; t < min(8, p.N - n); ++t)
                                 d16[n + t] = (uint16_t)((ww[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
                         }
                     }
@@ -410,7 +411,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // Split-K reduction: D[m,n] = sum over splits (fixed order) of ws[s][m][n].
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ ws, int splits, int64_t M,
                                                             int64_t N, int64_t ldw, void* __restrict__ D,
-                                                            int64_t ldd, int out_f32)
+                                                            int64_t ldd, int out_f32, int vec_out)
 {
     const int64_t nq = (N + 3) >> 2;          // 4-column chunks per row
     const int64_t total = M * nq;
@@ -427,17 +428,17 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
         const float v[4] = {s.x, s.y, s.z, s.w};
         if (out_f32) {
             float* d = reinterpret_cast<float*>(D) + m * ldd + n;
-            if (n + 4 <= N) *reinterpret_cast<float4*>(d) = s;
-            else for (int t = 0; t < N - n; ++t) d[t] = v[t];
+            if (vec_out && n + 4 <= N) *reinterpret_cast<float4*>(d) = s;
+            else for (int t = 0; t < (int)((N - n) < 4 ? (N - n) : 4); ++t) d[t] = v[t];
         } else {
             __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(D) + m * ldd + n;
             const uint32_t lo = cvt_bf16x2(s.x, s.y), hi = cvt_bf16x2(s.z, s.w);
-            if (n + 4 <= N) {
+            if (vec_out && n + 4 <= N) {
                 *reinterpret_cast<uint2*>(d) = make_uint2(lo, hi);
             } else {
                 const uint32_t ww[2] = {lo, hi};
                 uint16_t* d16 = reinterpret_cast<uint16_t*>(d);
-                for (int t = 0; t < N - n; ++t) d16[t] = (uint16_t)((ww[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+                for (int t = 0; t < (int)((N - n) < 4 ? (N - n) : 4); ++t) d16[t] = (uint16_t)((ww[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
             }
         }
     }

@@ -1,0 +1,114 @@
+"""Single-kernel cases for profiling (ncu) and per-kernel timing.
+
+  python -m fp8_block_scaled_11_b200.profile_cases <case> [--reps R] [--time]
+
+Cases (seeded inputs of the workloads, operands prepared before the loop so
+only the named kernel runs R times):
+  gemm_fwd     Llama4 forward GEMM 16640 x 5120 x 8192, 1x128 x 128x128, bf16 out
+  gemm_wgrad   Llama4 wgrad GEMM 5120 x 8192 x 16640, 1x128 x 1x128, bf16 out
+  gemm_tensor  16640 x 5120 x 8192 per-tensor scales, bf16 out
+  gemm_longk   256 x 512 x 128128 (k_blocks 1001), 1x128 x 128x128, split-K, bf16 out
+  quant_rows   1x128 quantization of a 32768 x 32768 bf16 matrix
+  quant_cols   1x128 along rows (transposed output) of a 16640 x 8192 bf16 matrix
+  quant_tile   128x128 quantization (with transposed copy) of a 32768 x 32768 bf16 matrix
+With --time, each launch is timed with CUDA events and the mean is printed.
+"""
+from __future__ import annotations
+
+import argparse
+import sys
+
+import torch
+
+from . import inputs, ops
+
+
+def _gemm_case(name):
+    M = inputs.LLAMA4_M
+    if name in ("gemm_fwd", "gemm_tensor"):
+        x, W, _ = inputs.llama4(5120, 8192)
+        x, W = x.cuda(), W.cuda()
+        if name == "gemm_fwd":
+            qa, sa = ops.fp8_quant_1x128(x)
+            qb, sb, _, _ = ops.fp8_quant_128x128(W)
+            mode = ops.SCALE_BLOCK_1x128_128x128
+        else:
+            qa, sa = ops.fp8_quant_tensor(x)
+            qb, sb = ops.fp8_quant_tensor(W)
+            mode = ops.SCALE_TENSOR
+        out = torch.empty((M, 5120), dtype=torch.bfloat16, device="cuda")
+        flops = 2.0 * M * 5120 * 8192
+    elif name == "gemm_wgrad":
+        x, _, dy = inputs.llama4(5120, 8192)
+        qa, sa = ops.fp8_quant_1x128(dy.cuda(), transpose_out=True)
+        qb, sb = ops.fp8_quant_1x128(x.cuda(), transpose_out=True)
+        mode = ops.SCALE_BLOCK_1x128_1x128
+        out = torch.empty((5120, 8192), dtype=torch.bfloat16, device="cuda")
+        flops = 2.0 * M * 5120 * 8192
+    else:
+        goT, x = inputs.long_k(128128)
+        qa, sa = ops.fp8_quant_1x128(goT.cuda())
+        _, _, qb, sb = ops.fp8_quant_128x128(x.cuda(), want_q=False, want_qt=True)
+        mode = ops.SCALE_BLOCK_1x128_128x128
+        out = torch.empty((256, 512), dtype=torch.bfloat16, device="cuda")
+        flops = 2.0 * 256 * 512 * 128128
+    ws = ops.fp8_scaled_gemm_workspace_size(qa.shape[0], qb.shape[0], qa.shape[1], mode)
+    wsb = torch.empty((max(ws, 16),), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    return (lambda: ops.fp8_scaled_gemm(qa, qb, sa, sb, mode, out=out, workspace=wsb)), flops, "TFLOP/s"
+
+
+def _quant_case(name):
+    if name == "quant_cols":
+        x = inputs.llama4(5120, 8192)[0].cuda()
+        q, s = ops.fp8_quant_1x128(x, transpose_out=True)
+        nbytes = x.numel() * 3 + 4 * s.numel()
+        fn = lambda: ops.fp8_quant_1x128(x, transpose_out=True, q=q, scale_inv=s)
+    else:
+        x = inputs.quant_sweep(32768).cuda()
+        if name == "quant_rows":
+            q, s = ops.fp8_quant_1x128(x)
+            nbytes = x.numel() * 3 + 4 * s.numel()
+            fn = lambda: ops.fp8_quant_1x128(x, q=q, scale_inv=s)
+        else:
+            out = ops.fp8_quant_128x128(x, want_q=True, want_qt=True)
+            nbytes = x.numel() * 4 + 8 * out[1].numel()
+            fn = lambda: ops.fp8_quant_128x128(x, want_q=True, want_qt=True, out=out)
+    torch.cuda.synchronize()
+    return fn, nbytes, "GB/s"
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case")
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--time", action="store_true")
+    a = ap.parse_args(argv)
+    if a.case.startswith("gemm"):
+        fn, work, unit = _gemm_case(a.case)
+    else:
+        fn, work, unit = _quant_case(a.case)
+    fn()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * a.reps)]
+    for i in range(a.reps):
+        if a.time:
+            ev[2 * i].record()
+        fn()
+        if a.time:
+            ev[2 * i + 1].record()
+    torch.cuda.synchronize()
+    st = ops.fp8bs_check_device_error()
+    if st != 0:
+        print(ops.fp8bs_status_string(st), file=sys.stderr)
+        return 1
+    if a.time:
+        ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(a.reps)]
+        mean = sum(ms) / len(ms)
+        rate = work / (mean * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+        print(f"{a.case}: {mean * 1e3:.1f} us/launch (mean of {a.reps}), {rate:.1f} {unit}")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

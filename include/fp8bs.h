@@ -182,9 +182,11 @@ fp8bs_status fp8_quant_rowwise(const void* x, fp8bs_dtype xt, int64_t rows, int6
  *            deterministic.
  * Any M, N >= 1 and any K >= 16 with K % 16 == 0 (any number of K blocks;
  * a ragged last K block contributes its valid columns only).
- * Alignment: A, Bt, D, scale_a, scale_b, workspace 16-byte aligned; lda, ldb
- * multiples of 16; ldd*sizeof(out) a multiple of 16; ld_sa, ld_sb % 4 == 0 for
- * the block modes.
+ * Alignment: A, Bt, scale_a, scale_b, workspace 16-byte aligned; lda, ldb
+ * multiples of 16; ld_sa, ld_sb % 4 == 0 for the block modes; D aligned to its
+ * element size.  Any ldd >= N works; when D is 16-byte aligned and
+ * ldd*sizeof(out) is a multiple of 16 the output is written in 16-byte
+ * chunks, otherwise element by element.
  */
 size_t fp8_scaled_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8bs_scale_mode mode);
 fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K,

@@ -103,8 +103,8 @@ def test_gemm_validation(L):
     assert gemm(L, mode=2, ldsb=1) == INVALID            # ld_sb < ceil(N/128)
     assert gemm(L, ldsa=258) == ALIGN
     assert gemm(L, lda=264) == ALIGN
-    assert gemm(L, ldd=260, od=0) == ALIGN               # 520 B row pitch
-    assert gemm(L, D=BAD) == ALIGN
+    assert gemm(L, D=BAD) == ALIGN                       # not element-aligned
+    assert gemm(L, D=GOOD + 2, od=1) == ALIGN            # fp32 output needs 4-byte alignment
     assert gemm(L, sa=GOOD + 4) == ALIGN
 
 

@@ -143,7 +143,7 @@ def test_special_values():
     """amax exactly 448 (s = 1), negative underflow to -0 (0x80), all-zero
     groups, subnormal-producing values, and huge dynamic range in one group."""
     C = 512
-    x = inputs.random_matrix(8, C, seed=5, dtype=torch.float32)
+    x = inputs.random_matrix(16, C, seed=5, dtype=torch.float32)
     x[0, :128] = 0.0
     x[0, 128:256] = -0.0
     x[1, :] = torch.linspace(-448, 448, C)
