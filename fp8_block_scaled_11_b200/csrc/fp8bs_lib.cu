@@ -445,3 +445,66 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- per-tensor quantization without allocation
+//
+// fp8_quant_tensor needs a small device workspace for its per-CTA amax
+// partials, which the caller allocates.  fp8_quant_tensor_noalloc runs the same
+// two kernels with that scratch taken from a fixed array compiled into the
+// library instead, so a caller that cannot allocate device memory at the point
+// of the call still gets the quantization.  The array is 16 KB per GPU, held
+// from the library's load on that GPU until the process exits.
+
+namespace {
+constexpr int kNoAllocPartials = 4096;                  // floats of scratch (16 KB)
+constexpr int64_t kNoAllocElemsPerPartial = 65536;      // elements reduced per amax CTA
+constexpr int64_t kNoAllocMaxElems = (int64_t)kNoAllocPartials * kNoAllocElemsPerPartial;
+float* g_noalloc_scratch[kMaxDevices] = {nullptr};      // device address of the array, per device
+std::mutex g_noalloc_mutex;
+}  // namespace
+
+// The scratch itself.  In host code this name is only a host-side stand-in for
+// the symbol: its device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocPartials];
+
+extern "C" fp8bs_status fp8_quant_tensor_noalloc(const void* x, fp8bs_dtype xt, int64_t n, uint8_t* q,
+                                                 float* scale_inv, cudaStream_t stream)
+{
+    if (!valid_dtype(xt)) return FP8BS_ERR_UNSUPPORTED;
+    if (x == nullptr || q == nullptr || scale_inv == nullptr || n < 1) return FP8BS_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scale_inv) & 3) || n % 16)
+        return FP8BS_ERR_ALIGNMENT;
+    if (n > kNoAllocMaxElems) return FP8BS_ERR_WORKSPACE;   // the built-in scratch covers at most this many
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP8BS_ERR_CUDA;
+    if (g_noalloc_scratch[dev] == nullptr) {
+        // one-time set-up per device, with that device current
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        if (g_noalloc_scratch[dev] == nullptr) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || p == nullptr) return FP8BS_ERR_CUDA;
+            g_noalloc_scratch[dev] = static_cast<float*>(p);
+        }
+    }
+    float* partial = g_noalloc_scratch[dev];
+    // every partial slot the second kernel reads is written by the first one in
+    // this same call, so nothing left by an earlier call needs clearing
+    const int parts = (int)std::max<int64_t>(1, cdiv(n, kNoAllocElemsPerPartial));
+    if (parts > kNoAllocPartials) return FP8BS_ERR_WORKSPACE;
+    const int64_t chunks = n / 8;
+    if (xt == FP8BS_BF16) {
+        tensor_amax_kernel<__nv_bfloat16><<<parts, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), n, partial);
+        auto k = tensor_quant_kernel<__nv_bfloat16>;
+        int g = persistent_grid(d, 6, k, cdiv(chunks, 256));
+        k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), n, partial, parts, q, scale_inv);
+    } else {
+        tensor_amax_kernel<float><<<parts, 256, 0, stream>>>(static_cast<const float*>(x), n, partial);
+        auto k = tensor_quant_kernel<float>;
+        int g = persistent_grid(d, 7, k, cdiv(chunks, 256));
+        k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), n, partial, parts, q, scale_inv);
+    }
+    return launch_status();
+}

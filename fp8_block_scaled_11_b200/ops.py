@@ -226,3 +226,21 @@ def fp8bs_status_string(status: int) -> str:
 def fp8bs_check_device_error(stream: Optional[torch.cuda.Stream] = None) -> int:
     s = stream if stream is not None else torch.cuda.current_stream()
     return int(lib().fp8bs_check_device_error(ctypes.c_void_p(s.cuda_stream)))
+
+
+def fp8_quant_tensor_noalloc(x: torch.Tensor, q: Optional[torch.Tensor] = None,
+                             scale_inv: Optional[torch.Tensor] = None):
+    """Per-tensor quantization through fp8_quant_tensor_noalloc (no workspace:
+    the library uses its built-in 16 KB scratch).  Returns (q, scale_inv[1]);
+    pass preallocated q / scale_inv to keep the call itself allocation-free."""
+    L = lib()
+    fn = L.fp8_quant_tensor_noalloc
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    if q is None:
+        q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale_inv is None:
+        scale_inv = torch.empty((1,), dtype=torch.float32, device=x.device)
+    _check("fp8_quant_tensor_noalloc", fn(x.data_ptr(), _dtype_code(x), x.numel(), q.data_ptr(),
+                                          scale_inv.data_ptr(), _stream(x)))
+    return q, scale_inv

@@ -140,6 +140,33 @@ fp8bs_status fp8_quant_tensor(const void* x, fp8bs_dtype xt, int64_t n, uint8_t*
                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * fp8_quant_tensor_noalloc -- fp8_quant_tensor for callers that cannot
+ * allocate device memory.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot call cudaMalloc (or any allocator) where they quantize -- for
+ * example a plugin whose host framework hands it no workspace, or code that
+ * must not trigger an allocation's implicit device synchronization or grow
+ * its memory footprint.  Same arguments, result and alignment rules as
+ * fp8_quant_tensor, minus the workspace: its amax scratch is a fixed 16 KB
+ * array compiled into the library, which every GPU that loads the library
+ * holds until the process exits.  This entry point allocates nothing.
+ *
+ * Limit: n <= 268435456 (2^28) elements; larger n returns FP8BS_ERR_WORKSPACE
+ * without launching anything.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.
+ * Sharing: all calls on a device share the one array.  Calls whose kernels
+ * overlap on the GPU (e.g. issued on different streams without ordering)
+ * race on it and may return wrong scales; order them on one stream or with
+ * events.  Nothing needs clearing between calls: every scratch slot a call
+ * reads was written earlier in the same call.
+ */
+fp8bs_status fp8_quant_tensor_noalloc(const void* x, fp8bs_dtype xt, int64_t n, uint8_t* q, float* scale_inv,
+                                      cudaStream_t stream);
+
+/*
  * fp8_quant_rowwise -- dynamic quantization with one scale per row.
  *
  * Defined by: the rowwise variant of scaled_mm (pytorch/pytorch issue #159940,
