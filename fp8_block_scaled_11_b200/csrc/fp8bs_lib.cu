@@ -147,7 +147,7 @@ int num_sms_current()
 
 template <int MODE>
 fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA,
-                                const CUtensorMap& tSB, const GemmParams& p, cudaStream_t stream)
+                         const CUtensorMap& tSB, const GemmParams& p, cudaStream_t stream)
 {
     auto k = gemm_fp8_kernel<MODE>;
     if (!d->gemm_attr_set[MODE]) {
@@ -156,7 +156,7 @@ fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap
         d->gemm_attr_set[MODE] = true;
     }
     const int grid = (int)std::min<int64_t>(p.num_units, d->num_sms);
-    k<<<grid, kThreads, SmemLayout::alloc, stream>>>(tA, tB, tSA, tSB, p);
+    k<<<grid, EpiCfg<MODE>::threads, SmemLayout::alloc, stream>>>(tA, tB, tSA, tSB, p);
     return launch_status();
 }
 
@@ -227,7 +227,7 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
             k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
         }
     } else {
-        const int64_t ctas = cdiv(rows, 128) * cdiv(cols, 64);
+        const int64_t ctas = cdiv(rows, 128) * cdiv(cols, 128);
         if (xt == FP8BS_BF16) {
             auto k = quant_1x128_cols_kernel<__nv_bfloat16>;
             int g = persistent_grid(d, 2, k, ctas);

@@ -8,21 +8,23 @@
 // per-tensor / rowwise recipes of ROCm/aiter issue #1765 and pytorch/pytorch
 // issue #159940.
 //
-// Structure (one persistent CTA per SM, 320 threads = 10 warps):
-//   warp 0      TMA producer: for each K-block, one 128x128 tile of A and one
-//               256x128 tile of B (bytes, 128-byte swizzle) into an S-stage
-//               shared-memory ring; per-K-block scale vectors into a separate
-//               ring (they are consumed later, by the epilogue).
-//   warp 1      TMEM owner + MMA issuer: one elected thread issues four
-//               tcgen05.mma (128x256x32, e4m3 x e4m3 -> fp32) per K-block into
-//               one of two 256-column TMEM accumulators, and commits the smem
-//               stage back to the producer when the MMAs have read it.
-//   warps 2-9   epilogue / promotion: per accumulation group (one K-block for
-//               the block recipes; the whole K range for tensor/rowwise) they
-//               tcgen05.ld the partial sums, multiply by the scale product and
-//               add into fp32 registers (packed f32x2 FMA), then release the
-//               TMEM buffer so the MMA of group g+2 can start.  At the end of
-//               a tile the registers are converted and stored.
+// One persistent CTA per SM computes 128 x 256 output tiles:
+//   warp 0      TMA producer: per K-block one 128x128 tile of A and one
+//               256x128 tile of B^T (bytes, 128-byte swizzle) into a 4-stage
+//               shared-memory ring, and the K-block's scale vectors into a
+//               separate ring (they are read later, by the promotion warps).
+//   warp 1      TMEM allocation; lane 0 issues four tcgen05.mma (128x256x32,
+//               e4m3 x e4m3 -> fp32) per K-block into one of two 256-column
+//               TMEM accumulators and commits the accumulator and the smem
+//               stage when the MMAs complete.
+//   warps 2..   promotion / epilogue (8 warps, or 16 for the 1x128 x 1x128
+//               recipe whose per-column scales double the per-element work):
+//               per accumulation group (one K-block for the block recipes; the
+//               whole K range for tensor/rowwise) they tcgen05.ld the partial
+//               sums, multiply by the scale product and add into fp32 registers
+//               (packed f32x2 FMA), then release the TMEM buffer so the MMA of
+//               group g+2 can start.  At the end of a tile the registers are
+//               converted and stored.
 // The per-K-block promotion keeps every partial sum in fp32 with the exact
 // scale product of its block, which is what makes any number of K blocks
 // (1000, 1001, 1002, ...) safe: scale indexing is kb*ld + i with no padding
@@ -41,34 +43,45 @@
 
 namespace fp8bs {
 
-constexpr int kBM = 128;             // tile rows (A rows, TMEM lanes)
-constexpr int kBN = 256;             // tile cols (B rows, TMEM columns per accumulator)
-constexpr int kBK = 128;             // K-block = scale block = one 128-byte swizzle row
-constexpr int kStages = 4;           // A/B smem ring depth
-constexpr int kScaleStages = 8;      // scale ring depth (>= kStages + 2 + 1)
-constexpr int kThreads = 320;
-constexpr int kEpiWarps = 8;
-constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
+constexpr int kBM = 128;                        // tile rows (TMEM lanes)
+constexpr int kBN = 256;                        // tile columns (TMEM columns per accumulator)
+constexpr int kBK = 128;                        // K-block = scale block = one 128-byte swizzle row
+constexpr uint32_t kTmemCols = 512;             // all of TMEM
+constexpr int kTmemBufs = kTmemCols / kBN;      // two accumulators in flight
+constexpr int kStages = 4;                      // A/B smem ring depth
+constexpr int kScaleStages = kStages + kTmemBufs + 2;   // scale ring depth (> kStages + kTmemBufs)
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // pipeline waits
 constexpr uint64_t kDrainLimitNs = 1000000000ull;  // exit-time waits for work in flight
 
-constexpr uint32_t kATileBytes = kBM * kBK;            // 16 KB
-constexpr uint32_t kBTileBytes = kBN * kBK;            // 32 KB
-constexpr uint32_t kScaleEntryBytes = (kBM + kBN) * 4; // sa[128] then sb[256]
+constexpr uint32_t kATileBytes = kBM * kBK;             // 16 KB
+constexpr uint32_t kBTileBytes = kBN * kBK;             // 32 KB
+constexpr uint32_t kScaleEntryBytes = (kBM + kBN) * 4;  // sa[128] then sb[256]
 
 struct SmemLayout {
     static constexpr uint32_t a_off = 0;
     static constexpr uint32_t b_off = a_off + kStages * kATileBytes;
     static constexpr uint32_t sc_off = b_off + kStages * kBTileBytes;
     static constexpr uint32_t bar_off = sc_off + kScaleStages * kScaleEntryBytes;
-    // barriers: ab_full[S], ab_empty[S], sc_full[SS], sc_empty[SS], tm_full[2], tm_empty[2], drain
-    static constexpr uint32_t n_bars = 2 * kStages + 2 * kScaleStages + 4 + 1;
+    // ab_full[S], ab_empty[S], sc_full[SS], sc_empty[SS], tm_full[2], tm_empty[2], drain
+    static constexpr uint32_t n_bars = 2 * kStages + 2 * kScaleStages + 2 * kTmemBufs + 1;
     static constexpr uint32_t misc_off = bar_off + n_bars * 8;
     static constexpr uint32_t total = misc_off + 16;
     static constexpr uint32_t alloc = total + 1024;     // slack to align the base to 1024 B
 };
 
 enum GemmMode : int { kModeTensor = 0, kModeRowwise = 1, kModeBlock128 = 2, kModeBlock1x128 = 3 };
+
+// Promotion-warp configuration per recipe (measured on B200: the 1x128 x
+// 128x128 recipe is fastest with 8 warps loading one 16-column TMEM chunk at a
+// time, the 1x128 x 1x128 recipe with 16 warps keeping two chunks in flight).
+template <int MODE>
+struct EpiCfg {
+    static constexpr int warps = MODE == kModeBlock1x128 ? 16 : 8;
+    static constexpr bool single_buf = MODE == kModeBlock128;
+    static constexpr int threads = 64 + 32 * warps;
+    static constexpr int cols = kBN * 4 / warps;        // accumulator columns per thread
+    static constexpr int chunks = cols / 16;            // 16-column TMEM loads per group
+};
 
 struct GemmParams {
     int32_t M, N, K;
@@ -106,11 +119,15 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int64_t u, int&
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(EpiCfg<MODE>::threads, 1)
 gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                 const GemmParams p)
 {
+    using E = EpiCfg<MODE>;
+    constexpr int kEpiWarps = E::warps;
+    constexpr int kColsPerThread = E::cols;
+    constexpr int kChunks = E::chunks;
     constexpr bool kPromote = (MODE == kModeBlock128 || MODE == kModeBlock1x128);
     constexpr bool kScaleRing = (MODE != kModeTensor);
     constexpr bool kColScales = (MODE == kModeBlock1x128 || MODE == kModeRowwise);
@@ -125,8 +142,8 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     auto sc_full = [&](int s) { return bars + 8u * (2 * kStages + s); };
     auto sc_empty = [&](int s) { return bars + 8u * (2 * kStages + kScaleStages + s); };
     auto tm_full = [&](int b) { return bars + 8u * (2 * kStages + 2 * kScaleStages + b); };
-    auto tm_empty = [&](int b) { return bars + 8u * (2 * kStages + 2 * kScaleStages + 2 + b); };
-    const uint32_t drain_bar = bars + 8u * (2 * kStages + 2 * kScaleStages + 4);
+    auto tm_empty = [&](int b) { return bars + 8u * (2 * kStages + 2 * kScaleStages + kTmemBufs + b); };
+    const uint32_t drain_bar = bars + 8u * (2 * kStages + 2 * kScaleStages + 2 * kTmemBufs);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + SmemLayout::misc_off);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc_off + 4);
 
@@ -141,7 +158,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             mbar_init(sc_full(s), 1);
             mbar_init(sc_empty(s), kEpiWarps);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kTmemBufs; ++b) {
             mbar_init(tm_full(b), 1);
             mbar_init(tm_empty(b), kEpiWarps);
         }
@@ -235,12 +252,19 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 int kb = kb0;
                 for (int g = 0; g < ngroups && ok; ++g) {
                     const int kb_end = kPromote ? kb + 1 : kb1;
+                    // The smem stage of the group's first K-block is normally
+                    // ready long before the TMEM buffer is free: wait for it
+                    // first, so that only the TMEM hand-off is on the critical path.
+                    if (!mbar_wait_bounded(ab_full(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     if (!mbar_wait_bounded(tm_empty(tb), tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + (uint32_t)(tb * kBN);
+                    const int kb_first = kb;         // its stage was waited for above
                     for (; kb < kb_end; ++kb) {
-                        if (!mbar_wait_bounded(ab_full(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-                        tc_fence_after();
+                        if (kb != kb_first) {
+                            if (!mbar_wait_bounded(ab_full(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                            tc_fence_after();
+                        }
                         const uint32_t a_addr = sbase + SmemLayout::a_off + stage * kATileBytes;
                         const uint32_t b_addr = sbase + SmemLayout::b_off + stage * kBTileBytes;
 #pragma unroll
@@ -251,12 +275,13 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                             umma_f8(d_tmem, adesc, bdesc, idesc, acc);
                         }
                         issued = true;
+                        // the accumulator hand-off is on the critical path: signal it first
+                        if (kb + 1 == kb_end) umma_commit(tm_full(tb));
                         umma_commit(ab_empty(stage));
                         if (++stage == kStages) { stage = 0; phase ^= 1u; }
                     }
                     if (!ok) break;
-                    umma_commit(tm_full(tb));
-                    if (++tb == 2) { tb = 0; tphase ^= 1u; }
+                    if (++tb == kTmemBufs) { tb = 0; tphase ^= 1u; }
                 }
             }
             if (!ok) give_up();
@@ -267,10 +292,10 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             }
         }
     } else {
-        // ------------------------------------------------------------ epilogue
-        const int e = warp - 2;                 // 0..7
+        // ------------------------------------------------------------ promotion / epilogue
+        const int e = warp - 2;                 // 0 .. kEpiWarps-1
         const int lq = warp & 3;                // TMEM lane quarter this warp may access
-        const int ch = e >> 2;                  // column half: 0 -> cols 0..127, 1 -> 128..255
+        const int col0 = (e >> 2) * kColsPerThread;   // this warp's columns within the tile
         const int row_in_tile = lq * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(lq * 32) << 16;
         int tb = 0;
@@ -285,16 +310,15 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             int tm, tn, kb0, kb1, split;
             decode_unit(p, u, tm, tn, kb0, kb1, split);
             const int ngroups = kPromote ? (kb1 - kb0) : 1;
-            float2 acc[64];
+            float2 acc[kColsPerThread / 2];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
+            for (int i = 0; i < kColsPerThread / 2; ++i) acc[i] = make_float2(0.f, 0.f);
 
             for (int g = 0; g < ngroups; ++g) {
                 // every lane waits; the outcome is made warp-uniform so that a
-                // lane-local timeout cannot leave a diverged warp at tcgen05.ld
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(tm_full(tb), tphase, abort_flag, kWaitLimitNs));
-                if (!ok) break;
-                tc_fence_after();
+                // lane-local timeout cannot leave a diverged warp at tcgen05.ld.
+                // The group's scales arrive long before its partial sums: read
+                // them first, so only the TMEM hand-off is on the critical path.
                 uint32_t sc_addr = 0;
                 float rowf = tensor_scale;
                 if (kScaleRing) {
@@ -304,23 +328,18 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     sc_addr = sbase + SmemLayout::sc_off + ss * kScaleEntryBytes;
                     rowf = sc[row_in_tile];
                     if (MODE == kModeBlock128) {
-                        const int off = ((tn * kBN) / 128) & 3;
-                        rowf *= sc[kBM + off + ch];
+                        const int nb0 = (tn * kBN) / 128;
+                        rowf *= sc[kBM + (tn * kBN + col0) / 128 - (nb0 & ~3)];
                     }
                 }
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(tm_full(tb), tphase, abort_flag, kWaitLimitNs));
+                if (!ok) break;
+                tc_fence_after();
                 const float2 rowf2 = make_float2(rowf, rowf);
-                const uint32_t tcol = tmem_base + lane_addr + (uint32_t)(tb * kBN + ch * 128);
-                // 8 chunks of 16 columns; the TMEM load of chunk c+1 is in flight
-                // while chunk c is promoted.
-                uint32_t rbuf[2][16];
-                tmem_ld_32x32b_x16(tcol, rbuf[0]);
-                tmem_ld_wait(rbuf[0]);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t (&r)[16] = rbuf[c & 1];
-                    if (c + 1 < 8) tmem_ld_32x32b_x16(tcol + (c + 1) * 16, rbuf[(c + 1) & 1]);
+                const uint32_t tcol = tmem_base + lane_addr + (uint32_t)(tb * kBN + col0);
+                auto promote = [&](int c, const uint32_t (&r)[16]) {
                     if (kColScales) {
-                        const uint32_t sb_addr = sc_addr + (uint32_t)((kBM + ch * 128 + c * 16) * 4);
+                        const uint32_t sb_addr = sc_addr + (uint32_t)((kBM + col0 + c * 16) * 4);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const float4 b4 = lds128(sb_addr + 16 * j);
@@ -331,11 +350,31 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
+                        for (int j = 0; j < 8; ++j)
                             acc[c * 8 + j] = ffma2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), rowf2, acc[c * 8 + j]);
-                        }
                     }
-                    if (c + 1 < 8) tmem_ld_wait(rbuf[(c + 1) & 1]);
+                };
+                if constexpr (E::single_buf) {
+                    // one 16-column load at a time; the sibling warps of the
+                    // SM sub-partition cover its latency
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c) {
+                        uint32_t r[16];
+                        tmem_ld_32x32b_x16(tcol + c * 16, r);
+                        tmem_ld_wait(r);
+                        promote(c, r);
+                    }
+                } else {
+                    // two 16-column loads in flight: chunk c+1 loads while c is promoted
+                    uint32_t rbuf[2][16];
+                    tmem_ld_32x32b_x16(tcol, rbuf[0]);
+                    tmem_ld_wait(rbuf[0]);
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c) {
+                        if (c + 1 < kChunks) tmem_ld_32x32b_x16(tcol + (c + 1) * 16, rbuf[(c + 1) & 1]);
+                        promote(c, rbuf[c & 1]);
+                        if (c + 1 < kChunks) tmem_ld_wait(rbuf[(c + 1) & 1]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -343,21 +382,21 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     mbar_arrive(tm_empty(tb));
                     if (kScaleRing) mbar_arrive(sc_empty(ss));
                 }
-                if (++tb == 2) { tb = 0; tphase ^= 1u; }
+                if (++tb == kTmemBufs) { tb = 0; tphase ^= 1u; }
                 if (kScaleRing) {
                     if (++ss == kScaleStages) { ss = 0; sphase ^= 1u; }
                 }
             }
             if (!ok) break;
 
-            // ---- store the tile: row m, columns n .. n+127 of this thread
+            // ---- store the tile: row m, this thread's kColsPerThread columns
             const int64_t m = (int64_t)tm * kBM + row_in_tile;
-            const int n_base = tn * kBN + ch * 128;
+            const int n_base = tn * kBN + col0;
             if (m < p.M) {
                 if (p.splits > 1) {
                     float* dst = p.ws + ((int64_t)split * p.M + m) * p.ldw;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
+                    for (int j = 0; j < kColsPerThread / 4; ++j) {
                         const int n = n_base + 4 * j;
                         if (n + 4 <= p.N) {
                             *reinterpret_cast<float4*>(dst + n) = make_float4(acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y);
@@ -369,7 +408,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 } else if (p.out_f32) {
                     float* dst = reinterpret_cast<float*>(p.D) + m * p.ldd;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
+                    for (int j = 0; j < kColsPerThread / 4; ++j) {
                         const int n = n_base + 4 * j;
                         if (p.vec_out && n + 4 <= p.N) {
                             *reinterpret_cast<float4*>(dst + n) = make_float4(acc[2 * j].x, acc[2 * j].y, acc[2 * j + 1].x, acc[2 * j + 1].y);
@@ -381,7 +420,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 } else {
                     __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + m * p.ldd;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
+                    for (int j = 0; j < kColsPerThread / 8; ++j) {
                         const int n = n_base + 8 * j;
                         const uint4 w = make_uint4(cvt_bf16x2(acc[4 * j].x, acc[4 * j].y),
                                                    cvt_bf16x2(acc[4 * j + 1].x, acc[4 * j + 1].y),
@@ -402,6 +441,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (!ok) give_up();
     }
 
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -265,3 +265,4 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b)
 }
 
 }  // namespace fp8bs
+

@@ -145,97 +145,125 @@ __global__ void __launch_bounds__(256) quant_1x128_rows_kernel(
 }
 
 // --------------------------------------------------------------------------
-// 1x128 groups along the ROWS, writing the quantized transpose.
-// Tile = 128 rows x 64 columns, staged through shared memory as fp32 (row
-// stride 65 words).  Pass 1: 4 threads per column reduce |x| over 128 rows.
-// Pass 2: each thread emits 16 consecutive output bytes (16 rows of one
-// column) of the transposed row; 64 scales per tile leave contiguously.
+// 128 x 128 tiles held as 8 x 8 register blocks.
+// Thread layout in a 256-thread CTA: warp w = (wr, wc) = (w >> 2, w & 3),
+// lane l = (ls, lg) = (l >> 3, l & 7); strip s = 4 wc + ls owns columns
+// [8s, 8s+8) of the tile, row group g = 8 wr + lg owns rows [8g, 8g+8).  For a
+// fixed row i a warp reads 8 rows x 64 contiguous bytes (bf16); for a fixed
+// column j it writes 4 transposed rows x 64 contiguous bytes, and row-major
+// output rows go out as 8 rows x 32 contiguous bytes: whole 32-byte sectors.
+// --------------------------------------------------------------------------
+template <typename T>
+struct Block8x8 {
+    Vec8<T> row[8];
+
+    __device__ __forceinline__ void load(const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ldx,
+                                         int64_t r0, int64_t c0)
+    {
+        const bool col_ok = c0 < cols;           // cols % 16 == 0: a strip of 8 is all-in or all-out
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (col_ok && r0 + i < rows) row[i].load(x + (r0 + i) * ldx + c0);
+            else row[i].zero();
+        }
+    }
+
+    __device__ __forceinline__ void col_absmax(float (&m)[8]) const
+    {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m[j] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float f[8];
+            row[i].get(f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m[j] = fmaxf(m[j], fabsf(f[j]));
+        }
+    }
+
+    // Column j quantized with scale s: the 8 bytes of rows 0..7 (row 0 lowest).
+    __device__ __forceinline__ uint2 quant_col(int j, float s) const
+    {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float f[8];
+            row[i].get(f);
+            v[i] = __fmul_rn(f[j], s);
+        }
+        const uint32_t w0 = cvt_e4m3x2(v[0], v[1]) | ((uint32_t)cvt_e4m3x2(v[2], v[3]) << 16);
+        const uint32_t w1 = cvt_e4m3x2(v[4], v[5]) | ((uint32_t)cvt_e4m3x2(v[6], v[7]) << 16);
+        return make_uint2(w0, w1);
+    }
+};
+
+__device__ __forceinline__ void block_coords(int& strip, int& group)
+{
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    strip = 4 * (w & 3) + (l >> 3);
+    group = 8 * (w >> 2) + (l & 7);
+}
+
+// --------------------------------------------------------------------------
+// 1x128 groups along the ROWS, writing the quantized transpose: the group of
+// output row c (input column c) is input rows [128 t, 128 t + 128).
+// Per column: max over the thread's 8 rows, over the 8 row groups of the warp
+// (lane shuffles), then over the two warps holding the tile's upper and lower
+// 64 rows (shared memory).  Output row c of the tile gets its 128 bytes from
+// 16 threads, 8 bytes each.
 // --------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(
     const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ldx,
     uint8_t* __restrict__ qt, int64_t ldq, float* __restrict__ sinv, int64_t ld_s)
 {
-    constexpr int TR = 128, TC = 64, PITCH = TC + 1;
-    __shared__ float tile[TR * PITCH];
-    __shared__ float s_scale[TC];
-    const int tid = threadIdx.x;
-    const int64_t tiles_r = (rows + TR - 1) / TR;
-    const int64_t tiles_c = (cols + TC - 1) / TC;
-    const int64_t ntiles = tiles_r * tiles_c;
+    __shared__ float s_half[2][128];           // column maxima of the tile's two 64-row halves
+    int strip, group;
+    block_coords(strip, group);
+    const int wr = (threadIdx.x >> 5) >> 2;
+    const int64_t tiles_c = (cols + 127) >> 7;
+    const int64_t ntiles = ((rows + 127) >> 7) * tiles_c;
 
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        const int64_t tr = t / tiles_c;
-        const int64_t tc = t - tr * tiles_c;
-        const int64_t r0 = tr * TR, c0 = tc * TC;
-        // load: 128 rows x 8 chunks of 8 values = 1024 chunks, 4 per thread
-        {
-            Vec8<T> v[4];
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t r0 = (tr << 7) + 8 * group;
+        const int64_t c0 = (tc << 7) + 8 * strip;
+        Block8x8<T> blk;
+        blk.load(x, rows, cols, ldx, r0, c0);
+        float m[8];
+        blk.col_absmax(m);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int id = tid + 256 * j;
-                const int lr = id >> 3, lc = (id & 7) << 3;
-                const int64_t r = r0 + lr, c = c0 + lc;
-                if (r < rows && c < cols) v[j].load(x + r * ldx + c);
-                else v[j].zero();
-            }
+        for (int j = 0; j < 8; ++j) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int id = tid + 256 * j;
-                const int lr = id >> 3, lc = (id & 7) << 3;
-                float f[8];
-                v[j].get(f);
+            for (int o = 1; o <= 4; o <<= 1) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], o));
+        }
+        if ((threadIdx.x & 7) == 0) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) tile[lr * PITCH + lc + e] = f[e];
-            }
+            for (int j = 0; j < 8; ++j) s_half[wr][8 * strip + j] = m[j];
         }
         __syncthreads();
-        // column amax: thread -> column tid/4, rows (tid%4)*32 .. +32
-        {
-            const int lc = tid >> 2, part = tid & 3;
-            float m = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(tile[(part * 32 + i) * PITCH + lc]));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            if (part == 0) s_scale[lc] = scale_from_amax(m);
-        }
-        __syncthreads();
-        // emit: 64 columns x 8 chunks of 16 rows = 512 chunks, 2 per thread
+        float sc[8];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int id = tid + 256 * j;
-            const int lc = id & 63;          // consecutive threads: consecutive columns (bank-friendly)
-            const int ch = id >> 6;          // 16-row chunk
-            const int64_t c = c0 + lc, r = r0 + ch * 16;
-            if (c < cols && r < rows) {      // rows % 16 == 0: chunks are all-in or all-out
-                const float s = s_scale[lc];
-                uint32_t w[4];
+        for (int j = 0; j < 8; ++j)
+            sc[j] = scale_from_amax(fmaxf(s_half[0][8 * strip + j], s_half[1][8 * strip + j]));
+        if (c0 < cols && r0 < rows) {          // rows % 16 == 0: a group of 8 rows is all-in or all-out
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int rr = ch * 16 + k * 4;
-                    const uint32_t lo = cvt_e4m3x2(__fmul_rn(tile[(rr + 0) * PITCH + lc], s),
-                                                   __fmul_rn(tile[(rr + 1) * PITCH + lc], s));
-                    const uint32_t hi = cvt_e4m3x2(__fmul_rn(tile[(rr + 2) * PITCH + lc], s),
-                                                   __fmul_rn(tile[(rr + 3) * PITCH + lc], s));
-                    w[k] = lo | (hi << 16);
-                }
-                *reinterpret_cast<uint4*>(qt + c * ldq + r) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint2*>(qt + (c0 + j) * ldq + r0) = blk.quant_col(j, sc[j]);
         }
-        if (tid < TC) {
-            const int64_t c = c0 + tid;
-            if (c < cols) sinv[c + tr * ld_s] = __frcp_rn(s_scale[tid]);
+        if (group == 0 && c0 < cols) {
+            float* dst = sinv + c0 + tr * ld_s;
+            *reinterpret_cast<float4*>(dst) = make_float4(__frcp_rn(sc[0]), __frcp_rn(sc[1]), __frcp_rn(sc[2]), __frcp_rn(sc[3]));
+            *reinterpret_cast<float4*>(dst + 4) = make_float4(__frcp_rn(sc[4]), __frcp_rn(sc[5]), __frcp_rn(sc[6]), __frcp_rn(sc[7]));
         }
         __syncthreads();
     }
 }
 
 // --------------------------------------------------------------------------
-// 128x128 tiles.  One CTA (256 threads) per tile: the tile (up to 32 KB of
-// bf16) is held in registers, 8 chunks of 8 values per thread; block-wide
-// amax through warp shuffles + shared memory; quantized bytes stored row-wise
-// and, when requested, staged in shared memory and stored transposed.
+// 128x128 tiles: one CTA per tile, the tile in registers as 8x8 blocks, amax
+// over the tile (shuffles + shared memory), then row-major and/or transposed
+// bytes straight from registers.
 // --------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) quant_128x128_kernel(
@@ -243,33 +271,24 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(
     uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sinv, int64_t ld_s,
     uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sinvt, int64_t ld_st)
 {
-    constexpr int QP = 128 + 16;             // byte pitch of the staged tile
     __shared__ float s_warp[8];
-    __shared__ __align__(16) uint8_t s_q[128 * QP];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int strip, group;
+    block_coords(strip, group);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t tiles_c = (cols + 127) >> 7;
-    const int64_t tiles_r = (rows + 127) >> 7;
-    const int64_t ntiles = tiles_r * tiles_c;
+    const int64_t ntiles = ((rows + 127) >> 7) * tiles_c;
 
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
         const int64_t bi = t / tiles_c, bj = t - bi * tiles_c;
-        const int64_t r0 = bi << 7, c0 = bj << 7;
-        // chunk id = tid + 256*j: row id/16, column chunk id%16 -> a warp reads 2 full 128-wide rows
-        Vec8<T> v[8];
+        const int64_t r0 = (bi << 7) + 8 * group;
+        const int64_t c0 = (bj << 7) + 8 * strip;
+        Block8x8<T> blk;
+        blk.load(x, rows, cols, ldx, r0, c0);
+        float m8[8];
+        blk.col_absmax(m8);
+        float m = m8[0];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int id = tid + 256 * j;
-            const int64_t r = r0 + (id >> 4), c = c0 + ((id & 15) << 3);
-            if (r < rows && c < cols) v[j].load(x + r * ldx + c);
-            else v[j].zero();
-        }
-        float m = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float f[8];
-            v[j].get(f);
-            m = fmaxf(m, absmax8(f));
-        }
+        for (int j = 1; j < 8; ++j) m = fmaxf(m, m8[j]);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) s_warp[warp] = m;
@@ -278,41 +297,24 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(
 #pragma unroll
         for (int w = 1; w < 8; ++w) amax = fmaxf(amax, s_warp[w]);
         const float s = scale_from_amax(amax);
+        const bool in = c0 < cols && r0 < rows;    // rows, cols % 16 == 0: blocks are all-in or all-out
+        if (q != nullptr && in) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int id = tid + 256 * j;
-            const int lr = id >> 4, lc = (id & 15) << 3;
-            const int64_t r = r0 + lr, c = c0 + lc;
-            float f[8];
-            v[j].get(f);
-            const uint2 b = quant8(f, s);
-            if (q != nullptr && r < rows && c < cols) *reinterpret_cast<uint2*>(q + r * ldq + c) = b;
-            if (qt != nullptr) *reinterpret_cast<uint2*>(s_q + lr * QP + lc) = b;
+            for (int i = 0; i < 8; ++i) {
+                float f[8];
+                blk.row[i].get(f);
+                *reinterpret_cast<uint2*>(q + (r0 + i) * ldq + c0) = quant8(f, s);
+            }
         }
-        if (tid == 0) {
+        if (qt != nullptr && in) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint2*>(qt + (c0 + j) * ldqt + r0) = blk.quant_col(j, s);
+        }
+        if (threadIdx.x == 0) {
             const float rinv = __frcp_rn(s);
             if (q != nullptr) sinv[bi + bj * ld_s] = rinv;
             if (qt != nullptr) sinvt[bj + bi * ld_st] = rinv;
-        }
-        if (qt != nullptr) {
-            __syncthreads();
-            // transposed: output row (c0+lc) gets bytes r0..r0+127; 128 cols x 8 chunks of 16 = 1024, 4 per thread
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int id = tid + 256 * j;
-                const int lc = id & 127, ch = id >> 7;
-                const int64_t c = c0 + lc, r = r0 + ch * 16;
-                if (c < cols && r < rows) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int rr = ch * 16 + k * 4;
-                        w[k] = (uint32_t)s_q[(rr + 0) * QP + lc] | ((uint32_t)s_q[(rr + 1) * QP + lc] << 8) |
-                               ((uint32_t)s_q[(rr + 2) * QP + lc] << 16) | ((uint32_t)s_q[(rr + 3) * QP + lc] << 24);
-                    }
-                    *reinterpret_cast<uint4*>(qt + c * ldqt + r) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
         }
         __syncthreads();
     }

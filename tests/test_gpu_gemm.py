@@ -275,3 +275,12 @@ def test_llama4_fwd_bwd_workload(N, K):
     assert_bytes_equal(step.dytq[torch.as_tensor(rows_n, device="cuda")], qdyto, "dy^T_q rows")
     ref = oracle.gemm(qdyto, qxto, sdyto, sxto, oracle.SCALE_BLOCK_1x128_1x128)
     assert_bf16_close(dW[torch.as_tensor(rows_n, device="cuda")], ref, "wgrad")
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("M", [129, 256, 257, 384, 512])
+def test_gemm_pair_tiles(M, mode):
+    """Row counts above 128 run on CTA pairs (256-row tiles): full pairs, a
+    pair whose second CTA is partly or wholly past the last row."""
+    run_random(M, 512, 384, mode, torch.float32, seed=M + 3 * mode)
+    run_random(M, 264, 1024, mode, torch.bfloat16, seed=M + 5 * mode, guard=True)
