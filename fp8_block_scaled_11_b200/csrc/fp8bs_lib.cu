@@ -31,6 +31,8 @@ struct DeviceInfo {
     int* err_ptr = nullptr;
     bool gemm_attr_set[4] = {false, false, false, false};
     int quant_blocks[10] = {0};  // resident CTAs per SM, per quant kernel kind
+    bool tile_attr_set[4] = {false, false, false, false};
+    int tile_blocks[4] = {0};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -95,6 +97,25 @@ int persistent_grid(DeviceInfo* d, int kind, Kernel k, int64_t work_ctas)
     }
     const int64_t cap = (int64_t)d->quant_blocks[kind] * d->num_sms;
     return (int)std::max<int64_t>(1, std::min<int64_t>(cap, work_ctas));
+}
+
+// Persistent launch of a TMA-pipelined tile kernel: resident CTAs per SM (for
+// its dynamic shared memory) x SMs, capped by the number of tiles.
+template <typename Kernel, typename... Args>
+fp8bs_status launch_tile_kernel(DeviceInfo* d, int kind, Kernel k, uint32_t smem, int64_t tiles, cudaStream_t stream,
+                                Args... args)
+{
+    if (!d->tile_attr_set[kind]) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return FP8BS_ERR_CUDA;
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k, 256, smem) != cudaSuccess || nb < 1) nb = 1;
+        d->tile_blocks[kind] = nb;
+        d->tile_attr_set[kind] = true;
+    }
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)d->tile_blocks[kind] * d->num_sms));
+    k<<<grid, 256, smem, stream>>>(args...);
+    return launch_status();
 }
 
 // 2-D tensor map over a row-major matrix: inner dim `inner` elements, `outer`
@@ -228,15 +249,21 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
         }
     } else {
         const int64_t ctas = cdiv(rows, 128) * cdiv(cols, 128);
+        CUtensorMap map;
         if (xt == FP8BS_BF16) {
-            auto k = quant_1x128_cols_kernel<__nv_bfloat16>;
-            int g = persistent_grid(d, 2, k, ctas);
-            k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
+            if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, ldx * 2, 128, 128,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
+                return st;
+            st = launch_tile_kernel(d, 0, quant_1x128_cols_kernel<__nv_bfloat16>, QTile<__nv_bfloat16>::smem, ctas,
+                                    stream, map, rows, cols, q, ldq, scale_inv, ld_scale, d->err_ptr);
         } else {
-            auto k = quant_1x128_cols_kernel<float>;
-            int g = persistent_grid(d, 3, k, ctas);
-            k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
+            if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, x, cols, rows, ldx * 4, 128, 128,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
+                return st;
+            st = launch_tile_kernel(d, 1, quant_1x128_cols_kernel<float>, QTile<float>::smem, ctas, stream, map, rows,
+                                    cols, q, ldq, scale_inv, ld_scale, d->err_ptr);
         }
+        if (st != FP8BS_OK) return st;
     }
     return launch_status();
 }
@@ -262,18 +289,22 @@ fp8bs_status fp8_quant_128x128(const void* x, fp8bs_dtype xt, int64_t rows, int6
     fp8bs_status st = get_device(&d);
     if (st != FP8BS_OK) return st;
     const int64_t ctas = rb * cb;
+    CUtensorMap map;
     if (xt == FP8BS_BF16) {
-        auto k = quant_128x128_kernel<__nv_bfloat16>;
-        int g = persistent_grid(d, 4, k, ctas);
-        k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale,
-                                 q_t, ldq_t, scale_inv_t, ld_scale_t);
+        if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, ldx * 2, 128, 128,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
+            return st;
+        st = launch_tile_kernel(d, 2, quant_128x128_kernel<__nv_bfloat16>, QTile<__nv_bfloat16>::smem, ctas, stream,
+                                map, rows, cols, q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t, ld_scale_t,
+                                d->err_ptr);
     } else {
-        auto k = quant_128x128_kernel<float>;
-        int g = persistent_grid(d, 5, k, ctas);
-        k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale, q_t,
-                                 ldq_t, scale_inv_t, ld_scale_t);
+        if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, x, cols, rows, ldx * 4, 128, 128,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
+            return st;
+        st = launch_tile_kernel(d, 3, quant_128x128_kernel<float>, QTile<float>::smem, ctas, stream, map, rows, cols,
+                                q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t, ld_scale_t, d->err_ptr);
     }
-    return launch_status();
+    return st;
 }
 
 size_t fp8_quant_tensor_workspace_size(int64_t n)

@@ -87,9 +87,11 @@ __device__ __forceinline__ uint2 quant8(const float (&f)[8], float s)
 // 1x128 groups along the contiguous dimension.
 // Work item = 32 rows x one 128-column group, owned by one warp.  A half-warp
 // covers one row's group (16 lanes x 8 values); the warp walks 2 rows per step
-// in batches of 8 steps (8 x 16 B loads in flight per lane).  Each lane ends
-// up holding the scale of row (32*item + lane), so the 32 scales of the item
-// (adjacent in the column-major grid) leave in one coalesced 128-byte store.
+// in two batches of 8 steps (8 loads of 16 B in flight per lane).  A batch's
+// 16 row maxima are gathered so that lane L holds the amax of row L, each lane
+// computes one scale (one IEEE divide per row, not per lane) and the scales
+// are broadcast back by shuffles.  A batch's 16 reciprocal scales (adjacent in
+// the column-major grid) leave in one coalesced 64-byte store.
 // --------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) quant_1x128_rows_kernel(
@@ -110,63 +112,90 @@ __global__ void __launch_bounds__(256) quant_1x128_rows_kernel(
         const int64_t g = it - rb * groups;
         const int64_t c = (g << 7) + (hl << 3);
         const bool col_ok = c < cols;   // cols % 16 == 0: a chunk of 8 is all-in or all-out
-        float my_scale = 0.f;
+        // two batches of 8 steps (16 rows each): 8 loads of 16 B in flight per lane
 #pragma unroll
-        for (int batch = 0; batch < 2; ++batch) {
+        for (int b = 0; b < 2; ++b) {
             Vec8<T> v[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int64_t r = (rb << 5) + ((batch * 8 + i) << 1) + half;
+                const int64_t r = (rb << 5) + (b << 4) + (i << 1) + half;
                 if (col_ok && r < rows) v[i].load(x + r * ldx + c);
                 else v[i].zero();
             }
+            float my_amax = 0.f;        // lanes 0..15: amax of row (32 rb + 16 b + lane)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int step = batch * 8 + i;
-                const int64_t r = (rb << 5) + (step << 1) + half;
                 float f[8];
                 v[i].get(f);
                 float amax = absmax8(f);
 #pragma unroll
                 for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                const float s = scale_from_amax(amax);
-                if (col_ok && r < rows) {
-                    *reinterpret_cast<uint2*>(q + r * ldq + c) = quant8(f, s);
-                }
-                const float rinv = __frcp_rn(s);
-                // lane 2*step + h receives the scale of row 2*step + h
-                const float other = __shfl_sync(0xffffffffu, rinv, (lane & 1) << 4);
-                if ((lane >> 1) == step) my_scale = other;
+                // lane 2i + h receives the amax of row 2i + h of the batch (held by half-warp h)
+                const float other = __shfl_sync(0xffffffffu, amax, (lane & 1) << 4);
+                if ((lane >> 1) == i) my_amax = other;
             }
+            const float my_s = scale_from_amax(my_amax);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int64_t r = (rb << 5) + (b << 4) + (i << 1) + half;
+                const float s = __shfl_sync(0xffffffffu, my_s, 2 * i + half);
+                float f[8];
+                v[i].get(f);
+                if (col_ok && r < rows) *reinterpret_cast<uint2*>(q + r * ldq + c) = quant8(f, s);
+            }
+            const int64_t r = (rb << 5) + (b << 4) + lane;
+            if (lane < 16 && r < rows) sinv[r + g * ld_s] = __frcp_rn(my_s);
         }
-        const int64_t r = (rb << 5) + lane;
-        if (r < rows) sinv[r + g * ld_s] = my_scale;
     }
 }
 
 // --------------------------------------------------------------------------
-// 128 x 128 tiles held as 8 x 8 register blocks.
-// Thread layout in a 256-thread CTA: warp w = (wr, wc) = (w >> 2, w & 3),
-// lane l = (ls, lg) = (l >> 3, l & 7); strip s = 4 wc + ls owns columns
-// [8s, 8s+8) of the tile, row group g = 8 wr + lg owns rows [8g, 8g+8).  For a
-// fixed row i a warp reads 8 rows x 64 contiguous bytes (bf16); for a fixed
-// column j it writes 4 transposed rows x 64 contiguous bytes, and row-major
-// output rows go out as 8 rows x 32 contiguous bytes: whole 32-byte sectors.
+// 128 x 128 tiles through a TMA ring in shared memory.
+//
+// One elected thread keeps kQStages tiles (the CTA's next ones in grid-stride
+// order) in flight with 2-D bulk tensor loads into a ring of shared-memory
+// stages, one mbarrier per stage; all 256 threads then read the current tile
+// from shared memory as 8 x 8 blocks: warp w = (wr, wc) = (w >> 1, w & 1),
+// lane l = (lg, ls) = (l >> 3, l & 7); strip s = 8 wc + ls owns tile columns
+// [8s, 8s+8), row group g = 4 wr + lg owns rows [8g, 8g+8).  Each 8-lane
+// phase of a 16-byte shared load reads 128 contiguous bytes (no bank
+// conflicts); for a fixed column j a warp writes 8 transposed rows x 32
+// contiguous bytes, and for a fixed row i 4 rows x 64 contiguous bytes.
+// The stage is refilled as soon as every thread holds its block in registers
+// (the amax reduction's barrier), so the next loads overlap the compute.
 // --------------------------------------------------------------------------
+constexpr int kQStages = 3;
+constexpr uint64_t kQWaitLimitNs = 2000000000ull;
+
+template <typename T>
+struct QTile {
+    static constexpr uint32_t row_bytes = 128 * sizeof(T);
+    static constexpr uint32_t bytes = 128 * row_bytes;                  // 32 KB (bf16) / 64 KB (fp32)
+    static constexpr uint32_t bar_off = kQStages * bytes;
+    static constexpr uint32_t smem = bar_off + 8 * kQStages + 1024;     // + alignment slack
+};
+
+// 8 consecutive values of row r, columns [8s, 8s+8), from a staged tile.
+template <typename T>
+__device__ __forceinline__ void lds_vec8(const uint8_t* tile, int r, int s, Vec8<T>& v);
+
+template <>
+__device__ __forceinline__ void lds_vec8<__nv_bfloat16>(const uint8_t* tile, int r, int s, Vec8<__nv_bfloat16>& v)
+{
+    v.raw = *reinterpret_cast<const uint4*>(tile + r * QTile<__nv_bfloat16>::row_bytes + s * 16);
+}
+
+template <>
+__device__ __forceinline__ void lds_vec8<float>(const uint8_t* tile, int r, int s, Vec8<float>& v)
+{
+    const float4* p = reinterpret_cast<const float4*>(tile + r * QTile<float>::row_bytes + s * 32);
+    v.a = p[0];
+    v.b = p[1];
+}
+
 template <typename T>
 struct Block8x8 {
     Vec8<T> row[8];
-
-    __device__ __forceinline__ void load(const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ldx,
-                                         int64_t r0, int64_t c0)
-    {
-        const bool col_ok = c0 < cols;           // cols % 16 == 0: a strip of 8 is all-in or all-out
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (col_ok && r0 + i < rows) row[i].load(x + (r0 + i) * ldx + c0);
-            else row[i].zero();
-        }
-    }
 
     __device__ __forceinline__ void col_absmax(float (&m)[8]) const
     {
@@ -197,93 +226,153 @@ struct Block8x8 {
     }
 };
 
-__device__ __forceinline__ void block_coords(int& strip, int& group)
+// The shared pipeline of both tile kernels: grid-stride tiles, a kQStages
+// ring of TMA loads, and a callback per tile that receives the staged tile.
+// `process(tile_smem, tile_index, release)` must call release() once its
+// block is in registers (after a __syncthreads); release() refills the stage.
+template <typename T, typename Process>
+__device__ __forceinline__ void tile_pipeline(const CUtensorMap* map, int64_t ntiles, int64_t tiles_c, int* err,
+                                              Process&& process)
 {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    strip = 4 * (w & 3) + (l >> 3);
-    group = 8 * (w >> 2) + (l & 7);
+    extern __shared__ uint8_t qsmem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    auto full = [&](int st) { return sbase + QTile<T>::bar_off + 8u * st; };
+    __shared__ int s_abort;
+    __shared__ int s_fills[kQStages];                 // loads issued per stage (thread 0 only)
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kQStages; ++st) {
+            mbar_init(full(st), 1);
+            s_fills[st] = 0;
+        }
+        s_abort = 0;
+        fence_barrier_init();
+        prefetch_tensormap(map);
+    }
+    __syncthreads();
+    auto issue = [&](int64_t t, int st) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        ++s_fills[st];
+        mbar_arrive_expect_tx(full(st), QTile<T>::bytes);
+        tma_load_2d(sbase + st * QTile<T>::bytes, map, full(st), (int32_t)(tc * 128), (int32_t)(tr * 128));
+    };
+    // prologue: the first kQStages tiles of this CTA
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kQStages; ++st) {
+            const int64_t t = blockIdx.x + (int64_t)st * gridDim.x;
+            if (t < ntiles) issue(t, st);
+        }
+    }
+    int st = 0;
+    uint32_t phase = 0;
+    int64_t k = 0;                                    // this CTA's tile counter
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
+        bool ok = mbar_wait_bounded(full(st), phase, &s_abort, kQWaitLimitNs);
+        if (!__syncthreads_and(ok)) {
+            if (threadIdx.x == 0) { s_abort = 1; atomicOr(err, 1); }
+            break;
+        }
+        const int this_st = st;
+        auto release = [&]() {
+            const int64_t tn = t + (int64_t)kQStages * gridDim.x;
+            if (threadIdx.x == 0 && tn < ntiles) issue(tn, this_st);
+        };
+        process(sm + this_st * QTile<T>::bytes, t, release);
+        if (++st == kQStages) { st = 0; phase ^= 1u; }
+    }
+    // every issued load has landed before the CTA exits (immediate unless a
+    // wait gave up with loads still in flight)
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < kQStages; ++j)
+            if (s_fills[j] > 0) mbar_wait_bounded(full(j), (uint32_t)((s_fills[j] - 1) & 1), nullptr, kQWaitLimitNs / 2);
+    }
+    __syncthreads();
 }
 
-// --------------------------------------------------------------------------
+__device__ __forceinline__ void qblock_coords(int& strip, int& group, int& wr, int& wc)
+{
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    wr = w >> 1;
+    wc = w & 1;
+    strip = 8 * wc + (l & 7);
+    group = 4 * wr + (l >> 3);
+}
+
 // 1x128 groups along the ROWS, writing the quantized transpose: the group of
-// output row c (input column c) is input rows [128 t, 128 t + 128).
-// Per column: max over the thread's 8 rows, over the 8 row groups of the warp
-// (lane shuffles), then over the two warps holding the tile's upper and lower
-// 64 rows (shared memory).  Output row c of the tile gets its 128 bytes from
-// 16 threads, 8 bytes each.
-// --------------------------------------------------------------------------
+// output row c (input column c) is input rows [128 t, 128 t + 128).  Column
+// maxima: the thread's 8 rows, the warp's 4 row groups (shuffles), the 4
+// warps holding the tile's 32-row quarters (shared memory).
 template <typename T>
 __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(
-    const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ldx,
-    uint8_t* __restrict__ qt, int64_t ldq, float* __restrict__ sinv, int64_t ld_s)
+    const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
+    uint8_t* __restrict__ qt, int64_t ldq, float* __restrict__ sinv, int64_t ld_s, int* err)
 {
-    __shared__ float s_half[2][128];           // column maxima of the tile's two 64-row halves
-    int strip, group;
-    block_coords(strip, group);
-    const int wr = (threadIdx.x >> 5) >> 2;
+    __shared__ float s_part[4][128];
+    __shared__ __align__(16) float s_scale[128];
+    int strip, group, wr, wc;
+    qblock_coords(strip, group, wr, wc);
     const int64_t tiles_c = (cols + 127) >> 7;
     const int64_t ntiles = ((rows + 127) >> 7) * tiles_c;
-
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    tile_pipeline<T>(&map, ntiles, tiles_c, err, [&](const uint8_t* tile, int64_t t, auto&& release) {
         const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t r0 = (tr << 7) + 8 * group;
-        const int64_t c0 = (tc << 7) + 8 * strip;
         Block8x8<T> blk;
-        blk.load(x, rows, cols, ldx, r0, c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lds_vec8<T>(tile, 8 * group + i, strip, blk.row[i]);
         float m[8];
         blk.col_absmax(m);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-#pragma unroll
-            for (int o = 1; o <= 4; o <<= 1) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], o));
+            m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], 8));
+            m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], 16));
         }
-        if ((threadIdx.x & 7) == 0) {
+        if ((threadIdx.x & 31) < 8) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) s_half[wr][8 * strip + j] = m[j];
+            for (int j = 0; j < 8; ++j) s_part[wr][8 * strip + j] = m[j];
         }
         __syncthreads();
-        float sc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            sc[j] = scale_from_amax(fmaxf(s_half[0][8 * strip + j], s_half[1][8 * strip + j]));
-        if (c0 < cols && r0 < rows) {          // rows % 16 == 0: a group of 8 rows is all-in or all-out
+        release();
+        // one scale per output row (tile column): threads 0..127
+        if (threadIdx.x < 128) {
+            const int c = threadIdx.x;
+            const float sc = scale_from_amax(fmaxf(fmaxf(s_part[0][c], s_part[1][c]), fmaxf(s_part[2][c], s_part[3][c])));
+            s_scale[c] = sc;
+            const int64_t cg = (tc << 7) + c;
+            if (cg < cols) sinv[cg + tr * ld_s] = __frcp_rn(sc);
+        }
+        __syncthreads();
+        const float4 sa = *reinterpret_cast<const float4*>(&s_scale[8 * strip]);
+        const float4 sb = *reinterpret_cast<const float4*>(&s_scale[8 * strip + 4]);
+        const float sc[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+        const int64_t r0 = (tr << 7) + 8 * group;
+        const int64_t c0 = (tc << 7) + 8 * strip;
+        if (c0 < cols && r0 < rows) {          // rows, cols % 16 == 0: 8-blocks are all-in or all-out
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<uint2*>(qt + (c0 + j) * ldq + r0) = blk.quant_col(j, sc[j]);
         }
-        if (group == 0 && c0 < cols) {
-            float* dst = sinv + c0 + tr * ld_s;
-            *reinterpret_cast<float4*>(dst) = make_float4(__frcp_rn(sc[0]), __frcp_rn(sc[1]), __frcp_rn(sc[2]), __frcp_rn(sc[3]));
-            *reinterpret_cast<float4*>(dst + 4) = make_float4(__frcp_rn(sc[4]), __frcp_rn(sc[5]), __frcp_rn(sc[6]), __frcp_rn(sc[7]));
-        }
-        __syncthreads();
-    }
+        __syncthreads();                       // s_part / s_scale are rewritten by the next tile
+    });
 }
 
-// --------------------------------------------------------------------------
-// 128x128 tiles: one CTA per tile, the tile in registers as 8x8 blocks, amax
-// over the tile (shuffles + shared memory), then row-major and/or transposed
-// bytes straight from registers.
-// --------------------------------------------------------------------------
+// 128x128 tiles: amax over the tile (shuffles + shared memory), then
+// row-major and/or transposed bytes straight from registers.
 template <typename T>
 __global__ void __launch_bounds__(256) quant_128x128_kernel(
-    const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ldx,
+    const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
     uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sinv, int64_t ld_s,
-    uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sinvt, int64_t ld_st)
+    uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sinvt, int64_t ld_st, int* err)
 {
     __shared__ float s_warp[8];
-    int strip, group;
-    block_coords(strip, group);
+    int strip, group, wr, wc;
+    qblock_coords(strip, group, wr, wc);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t tiles_c = (cols + 127) >> 7;
     const int64_t ntiles = ((rows + 127) >> 7) * tiles_c;
-
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    tile_pipeline<T>(&map, ntiles, tiles_c, err, [&](const uint8_t* tile, int64_t t, auto&& release) {
         const int64_t bi = t / tiles_c, bj = t - bi * tiles_c;
-        const int64_t r0 = (bi << 7) + 8 * group;
-        const int64_t c0 = (bj << 7) + 8 * strip;
         Block8x8<T> blk;
-        blk.load(x, rows, cols, ldx, r0, c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lds_vec8<T>(tile, 8 * group + i, strip, blk.row[i]);
         float m8[8];
         blk.col_absmax(m8);
         float m = m8[0];
@@ -293,10 +382,13 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(
         for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) s_warp[warp] = m;
         __syncthreads();
+        release();
         float amax = s_warp[0];
 #pragma unroll
         for (int w = 1; w < 8; ++w) amax = fmaxf(amax, s_warp[w]);
         const float s = scale_from_amax(amax);
+        const int64_t r0 = (bi << 7) + 8 * group;
+        const int64_t c0 = (bj << 7) + 8 * strip;
         const bool in = c0 < cols && r0 < rows;    // rows, cols % 16 == 0: blocks are all-in or all-out
         if (q != nullptr && in) {
 #pragma unroll
@@ -316,8 +408,8 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(
             if (q != nullptr) sinv[bi + bj * ld_s] = rinv;
             if (qt != nullptr) sinvt[bj + bi * ld_st] = rinv;
         }
-        __syncthreads();
-    }
+        __syncthreads();                       // s_warp is rewritten by the next tile
+    });
 }
 
 // --------------------------------------------------------------------------
