@@ -37,10 +37,30 @@ UNIT = "TFLOP/s"
 PAGES_FP8_US = (7746.98, 7783.31)
 FP8_SPEC_TFLOPS = 4500.0
 
-# DRAM traffic of one GEMM launch from an ncu capture, keyed by the SHA-256 of
-# the kernel source it was taken on (profiles/ holds the summary).  A changed
-# kernel reports null until it is captured again.
-GEMM_TRAFFIC = {}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
+# GEMM launch of the (5120, 8192) layer (16640 x 5120 x 8192), from an ncu
+# capture, keyed by a hash of the kernel source it was taken on (the summary is
+# profiles/gemm_fp8_fwd_llama4.md).  A changed kernel reports null until it is
+# captured again.
+GEMM_TRAFFIC = {"1fed641ce1cd015a": 557.3e6}
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of per-rank timings (ms) across the process group;
+    identity on one rank.  Every rank must call it at the same point."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def throughput_tflops(world, flops_per_step_per_rank, steps, ms_max):
+    """Whole-job throughput under weak scaling: all ranks' flops over the
+    slowest rank's time."""
+    return world * flops_per_step_per_rank * steps / (ms_max * 1e-3) / 1e12
 
 
 def kernel_hash():
@@ -151,12 +171,11 @@ def run_gpu(args):
             if events is None:
                 st.run(x, W, dy)
             else:
-                e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                # events: before quantization, then before / after each GEMM
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
                 e[0].record(stream)
                 st.quantize(x, W, dy)
-                e[1].record(stream)
-                st.gemms()
-                e[2].record(stream)
+                st.gemms(mark=lambda i: e[1 + i].record(stream))
                 events.append((st, e))
 
     for _ in range(args.warmup):
@@ -184,19 +203,18 @@ def run_gpu(args):
     clocks = sampler.stop()
     ms_total = t0.elapsed_time(t1)
     quant_ms = sum(e[0].elapsed_time(e[1]) for _, e in events)
-    gemm_ms = sum(e[1].elapsed_time(e[2]) for _, e in events)
-    if world > 1:
-        tt = torch.tensor([ms_total, quant_ms, gemm_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total, quant_ms, gemm_ms = tt.tolist()
+    gemm_ms = sum(e[1].elapsed_time(e[4]) for _, e in events)
+    # the roofline launch: forward GEMM of the first layer shape
+    fwd_ms = sum(e[1].elapsed_time(e[2]) for st, e in events if st is steps[0])
+    ms_total, quant_ms, gemm_ms, fwd_ms = max_over_ranks([ms_total, quant_ms, gemm_ms, fwd_ms], world, "cuda")
 
     flops_step = sum(st.flops() for st in steps)
     qbytes_step = sum(st.quant_bytes() for st in steps)
     ms_step = ms_total / args.steps
-    value = world * flops_step * args.steps / (ms_total * 1e-3) / 1e12
-    gemm_tflops = flops_step * args.steps / (gemm_ms * 1e-3) / 1e12
-    gemm_launches = 3 * len(steps) * args.steps
-    gemm_avg_us = gemm_ms * 1e3 / gemm_launches
+    value = throughput_tflops(world, flops_step, args.steps, ms_total)
+    gemm_tflops = throughput_tflops(1, flops_step, args.steps, gemm_ms)
+    fwd_avg_us = fwd_ms * 1e3 / args.steps
+    fwd_tflops = steps[0].gemm_flops() / (fwd_avg_us * 1e-6) / 1e12
     quant_gbs = qbytes_step * args.steps / (quant_ms * 1e-3) / 1e9
 
     peaks, peak_src = measured_peaks()
@@ -234,14 +252,10 @@ def run_gpu(args):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            tt = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = tt.item()
+        e_ms = max_over_ranks([a.elapsed_time(b)], world, "cuda")[0]
         bi = sum(sum(t.numel() * t.element_size() for t in d) for d in host_in)
         bo = sum(sum(t.numel() * t.element_size() for t in o) for o in host_out)
-        e2e = {"value": round(world * flops_step * n_e2e / (e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+        e2e = {"value": round(throughput_tflops(world, flops_step, n_e2e, e_ms), 2), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": n_e2e,
                "path": "pinned host tensors -> ops (C ABI) -> pinned host tensors"}
 
@@ -272,12 +286,13 @@ def run_gpu(args):
             "gemm_ms_per_step": round(gemm_ms / args.steps, 4),
         },
         "roofline": {
-            "kernel": "gemm_fp8_kernel (6 launches per step)",
-            "bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
-            "frac": round(gemm_tflops / fp8_peak, 3), "traffic": tr,
+            "kernel": "gemm_fp8_kernel<1x128 x 128x128>, forward GEMM 16640 x 5120 x 8192 (bf16 out)",
+            "bound": "tensor", "achieved": round(fwd_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+            "frac": round(fwd_tflops / fp8_peak, 3), "traffic": tr,
+            "algorithmic_per_launch": f"{steps[0].gemm_flops():.4g} flop; 348.6 MB (operands + bf16 output)",
             "peak_source": f"2 x {'sustained' if sustained else 'burst'} bf16 of {peak_src} "
                            f"({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'fallback'}), fp8/bf16 ratio 2",
-            "avg_launch_us": round(gemm_avg_us, 1),
+            "avg_launch_us": round(fwd_avg_us, 1),
         },
         "clocks": clocks,
         "gpu_launches": Fp8LinearStep.LAUNCHES_PER_STEP * len(steps) * args.steps,

@@ -477,6 +477,32 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
 
 }  // extern "C"
 
+// ---------------------------------------------------------------- self-test of the device timeout path
+
+namespace {
+// One thread waits, with the library's bounded wait, on an mbarrier phase
+// that nothing will ever complete; when the limit runs out it raises the
+// error flag exactly as a pipeline kernel does, and returns.
+__global__ void selftest_wait_kernel(uint64_t limit_ns, int* err)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t a = smem_u32(&bar);
+    mbar_init(a, 1);
+    fence_barrier_init();
+    if (!mbar_wait_bounded(a, 0, nullptr, limit_ns)) atomicOr(err, 1);
+}
+}  // namespace
+
+extern "C" fp8bs_status fp8bs_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream)
+{
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return FP8BS_ERR_INVALID_ARG;
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+    selftest_wait_kernel<<<1, 1, 0, stream>>>(limit_ns, d->err_ptr);
+    return launch_status();
+}
+
 // ---------------------------------------------------------------- per-tensor quantization without allocation
 //
 // fp8_quant_tensor needs a small device workspace for its per-CTA amax

@@ -56,11 +56,18 @@ class Fp8LinearStep:
         ops.fp8_quant_1x128(dy, q=self.dyq, scale_inv=self.dys)
         ops.fp8_quant_1x128(dy, transpose_out=True, q=self.dytq, scale_inv=self.dyts)
 
-    def gemms(self):
+    def gemms(self, mark=None):
+        """The three GEMMs; `mark(i)` (optional) is called before GEMM i and
+        after the last one (i = 3), e.g. to record CUDA events between them."""
         B2, B3 = ops.SCALE_BLOCK_1x128_128x128, ops.SCALE_BLOCK_1x128_1x128
+        mark = mark or (lambda i: None)
+        mark(0)
         ops.fp8_scaled_gemm(self.xq, self.wq, self.xs, self.ws, B2, out=self.y, workspace=self.workspace)
+        mark(1)
         ops.fp8_scaled_gemm(self.dyq, self.wtq, self.dys, self.wts, B2, out=self.dx, workspace=self.workspace)
+        mark(2)
         ops.fp8_scaled_gemm(self.dytq, self.xtq, self.dyts, self.xts, B3, out=self.dW, workspace=self.workspace)
+        mark(3)
 
     def run(self, x: torch.Tensor, W: torch.Tensor, dy: torch.Tensor):
         self.quantize(x, W, dy)
@@ -68,7 +75,11 @@ class Fp8LinearStep:
         return self.y, self.dx, self.dW
 
     def flops(self) -> float:
-        return 3 * 2.0 * self.M * self.N * self.K
+        return 3 * self.gemm_flops()
+
+    def gemm_flops(self) -> float:
+        """Flops of each of the three GEMMs (they are equal: 2 M N K)."""
+        return 2.0 * self.M * self.N * self.K
 
     def quant_bytes(self) -> float:
         """Algorithmic HBM bytes of the five quantization launches: bf16 read +

@@ -236,6 +236,18 @@ const char* fp8bs_status_string(fp8bs_status s);
  */
 fp8bs_status fp8bs_check_device_error(cudaStream_t stream);
 
+/*
+ * fp8bs_selftest_wait_timeout -- exercises the device-side failure detection.
+ *
+ * Not part of the method: a self-test of the library's bounded device waits.
+ * Launches one thread that waits, with the same bounded wait the GEMM
+ * pipeline uses, on an mbarrier phase nothing completes.  After `limit_ns`
+ * (1 .. 10^10 ns) it sets the device error flag and returns; nothing faults or
+ * hangs, and the CUDA context stays usable.  A following
+ * fp8bs_check_device_error(stream) returns FP8BS_ERR_TIMEOUT (and clears it).
+ */
+fp8bs_status fp8bs_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
