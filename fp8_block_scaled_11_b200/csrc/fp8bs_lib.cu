@@ -429,9 +429,7 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
         if ((st = make_map(&tSA, f32, 4, scale_a, M, 1, (M * 4 + 15) & ~int64_t(15), kBM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
         if ((st = make_map(&tSB, f32, 4, scale_b, N, 1, (N * 4 + 15) & ~int64_t(15), kBN, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
         break;
-    case FP8BS_SCALE_BLOCK_1x128_128x128:
-        if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, kBM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
-        if ((st = make_map(&tSB, f32, 4, scale_b, Nb, Kb, ld_sb * 4, 4, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+    case FP8BS_SCALE_BLOCK_1x128_128x128:       // scales read directly by the promotion warps
         break;
     case FP8BS_SCALE_BLOCK_1x128_1x128:
         if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, kBM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
@@ -457,6 +455,8 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
     p.ldw = plan.ldw;
     p.sa = scale_a;
     p.sb = scale_b;
+    p.ld_sa = ld_sa;
+    p.ld_sb = ld_sb;
     p.err = d->err_ptr;
 
     switch (mode) {

@@ -96,8 +96,9 @@ struct GemmParams {
     int32_t vec_out;            // 1: D and ldd allow 16-byte row-chunk stores
     float* ws;                  // split-K partials [splits][M][ldw] fp32
     int64_t ldw;
-    const float* sa;            // tensor mode: scale pointers read directly
+    const float* sa;            // scale pointers read directly (tensor mode, 1x128 x 128x128 mode)
     const float* sb;
+    int64_t ld_sa, ld_sb;       // their leading dimensions (block modes)
     int* err;                   // library error flag
 };
 
@@ -129,7 +130,11 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     constexpr int kColsPerThread = E::cols;
     constexpr int kChunks = E::chunks;
     constexpr bool kPromote = (MODE == kModeBlock128 || MODE == kModeBlock1x128);
-    constexpr bool kScaleRing = (MODE != kModeTensor);
+    // The 1x128 x 128x128 recipe needs two scalars per thread and K-block:
+    // they are read straight from global memory (L2), prefetched two K-blocks
+    // ahead.  Per-column scales (rowwise, 1x128 x 1x128) go through a
+    // shared-memory ring filled by TMA.
+    constexpr bool kScaleRing = (MODE == kModeRowwise || MODE == kModeBlock1x128);
     constexpr bool kColScales = (MODE == kModeBlock1x128 || MODE == kModeRowwise);
     constexpr uint32_t kScaleTx = kBM * 4 + (kColScales ? kBN * 4 : 16);
 
@@ -226,7 +231,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     filled |= 1u << stage;
                     fill_par = (fill_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
-                    if (kPromote) ok = issue_scales(m0, n0, kb);
+                    if (kPromote && kScaleRing) ok = issue_scales(m0, n0, kb);
                 }
             }
             if (!ok) give_up();
@@ -314,26 +319,43 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
             for (int i = 0; i < kColsPerThread / 2; ++i) acc[i] = make_float2(0.f, 0.f);
 
+            // 1x128 x 128x128: this thread's row scale and its columns' block
+            // scale, for K-blocks kb0, kb0+1 (loaded now) and kb0+2.. (loaded
+            // two groups ahead, from L2)
+            const int64_t m_glob = (int64_t)tm * kBM + row_in_tile;
+            const bool row_ok = m_glob < p.M;
+            const int nb_glob = (tn * kBN + col0) / 128;
+            const bool nb_ok = nb_glob * 128 < p.N;     // columns past N are never stored
+            // raw values only: the product is formed when the group is promoted,
+            // so the loads stay in flight for two groups
+            auto load_scales = [&](int kb, float& a, float& b) {
+                if (MODE != kModeBlock128 || kb >= kb1 || !row_ok || !nb_ok) { a = b = 0.f; return; }
+                a = __ldg(p.sa + m_glob + (int64_t)kb * p.ld_sa);
+                b = __ldg(p.sb + nb_glob + (int64_t)kb * p.ld_sb);
+            };
+            float pa0, pb0, pa1, pb1;
+            load_scales(kb0, pa0, pb0);
+            load_scales(kb0 + 1, pa1, pb1);
+
             for (int g = 0; g < ngroups; ++g) {
-                // every lane waits; the outcome is made warp-uniform so that a
-                // lane-local timeout cannot leave a diverged warp at tcgen05.ld.
-                // The group's scales arrive long before its partial sums: read
-                // them first, so only the TMEM hand-off is on the critical path.
+                // Every lane waits.  A wait that gives up raises the abort flag
+                // and the warp carries on (no warp vote per K-block); the
+                // outcome is voted once per tile, below.
                 uint32_t sc_addr = 0;
                 float rowf = tensor_scale;
+                if (MODE == kModeBlock128) {
+                    rowf = pa0 * pb0;
+                    pa0 = pa1;
+                    pb0 = pb1;
+                    load_scales(kb0 + g + 2, pa1, pb1);
+                }
                 if (kScaleRing) {
-                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(sc_full(ss), sphase, abort_flag, kWaitLimitNs));
-                    if (!ok) break;
+                    if (!mbar_wait_bounded(sc_full(ss), sphase, abort_flag, kWaitLimitNs)) { ok = false; give_up(); }
                     const float* sc = reinterpret_cast<const float*>(smem + SmemLayout::sc_off + ss * kScaleEntryBytes);
                     sc_addr = sbase + SmemLayout::sc_off + ss * kScaleEntryBytes;
                     rowf = sc[row_in_tile];
-                    if (MODE == kModeBlock128) {
-                        const int nb0 = (tn * kBN) / 128;
-                        rowf *= sc[kBM + (tn * kBN + col0) / 128 - (nb0 & ~3)];
-                    }
                 }
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(tm_full(tb), tphase, abort_flag, kWaitLimitNs));
-                if (!ok) break;
+                if (!mbar_wait_bounded(tm_full(tb), tphase, abort_flag, kWaitLimitNs)) { ok = false; give_up(); }
                 tc_fence_after();
                 const float2 rowf2 = make_float2(rowf, rowf);
                 const uint32_t tcol = tmem_base + lane_addr + (uint32_t)(tb * kBN + col0);
@@ -376,8 +398,9 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         if (c + 1 < kChunks) tmem_ld_wait(rbuf[(c + 1) & 1]);
                     }
                 }
+                // the warp-collective tcgen05.wait::ld above leaves all lanes'
+                // loads complete: lane 0 may release the buffer
                 tc_fence_before();
-                __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(tm_empty(tb));
                     if (kScaleRing) mbar_arrive(sc_empty(ss));
@@ -387,6 +410,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     if (++ss == kScaleStages) { ss = 0; sphase ^= 1u; }
                 }
             }
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
 
             // ---- store the tile: row m, this thread's kColsPerThread columns
