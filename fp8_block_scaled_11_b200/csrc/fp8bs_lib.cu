@@ -31,8 +31,8 @@ struct DeviceInfo {
     int* err_ptr = nullptr;
     bool gemm_attr_set[4] = {false, false, false, false};
     int quant_blocks[10] = {0};  // resident CTAs per SM, per quant kernel kind
-    bool tile_attr_set[4] = {false, false, false, false};
-    int tile_blocks[4] = {0};
+    bool tile_attr_set[6] = {false, false, false, false, false, false};
+    int tile_blocks[6] = {0};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -266,6 +266,42 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
         if (st != FP8BS_OK) return st;
     }
     return launch_status();
+}
+
+fp8bs_status fp8_quant_1x128_dual(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                                  uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale, uint8_t* q_t,
+                                  int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t, cudaStream_t stream)
+{
+    if (!valid_dtype(xt)) return FP8BS_ERR_UNSUPPORTED;
+    if (x == nullptr || q == nullptr || scale_inv == nullptr || q_t == nullptr || scale_inv_t == nullptr ||
+        rows < 1 || cols < 1)
+        return FP8BS_ERR_INVALID_ARG;
+    if (ldx < cols || ldq < cols || ld_scale < rows || ldq_t < rows || ld_scale_t < cols) return FP8BS_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(scale_inv) || !aligned16(q_t) || !aligned16(scale_inv_t))
+        return FP8BS_ERR_ALIGNMENT;
+    if ((ldx * (int64_t)dtype_size(xt)) % 16 || ldq % 16 || ldq_t % 16 || ld_scale % 4 || ld_scale_t % 4 ||
+        rows % 16 || cols % 16)
+        return FP8BS_ERR_ALIGNMENT;
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+    const int64_t ctas = cdiv(rows, 128) * cdiv(cols, 128);
+    CUtensorMap map;
+    if (xt == FP8BS_BF16) {
+        if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, ldx * 2, 128, 128,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
+            return st;
+        st = launch_tile_kernel(d, 4, quant_1x128_dual_kernel<__nv_bfloat16>, QTile<__nv_bfloat16>::smem, ctas, stream,
+                                map, rows, cols, q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t, ld_scale_t,
+                                d->err_ptr);
+    } else {
+        if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, x, cols, rows, ldx * 4, 128, 128,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
+            return st;
+        st = launch_tile_kernel(d, 5, quant_1x128_dual_kernel<float>, QTile<float>::smem, ctas, stream, map, rows,
+                                cols, q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t, ld_scale_t, d->err_ptr);
+    }
+    return st;
 }
 
 fp8bs_status fp8_quant_128x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,

@@ -354,6 +354,94 @@ __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(
     });
 }
 
+// Both 1x128 directions from one read of the input.  A 128 x 128 tile holds
+// 128 whole row groups (1x128 along the columns) and 128 whole column groups
+// (1x128 along the rows), so one pass over the tile gives both sets of
+// maxima: column maxima as in quant_1x128_cols_kernel, row maxima over the
+// thread's 8 columns, the warp's 8 strips (shuffles) and the tile's two
+// 64-column halves (shared memory).  Outputs are byte-identical to the
+// row-direction and transposed column-direction launches.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_1x128_dual_kernel(
+    const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
+    uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sinv, int64_t ld_s,
+    uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sinvt, int64_t ld_st, int* err)
+{
+    __shared__ float s_cpart[4][128];                 // column maxima per 32-row quarter
+    __shared__ float s_rpart[2][128];                 // row maxima per 64-column half
+    __shared__ __align__(16) float s_cscale[128];
+    __shared__ float s_rscale[128];
+    int strip, group, wr, wc;
+    qblock_coords(strip, group, wr, wc);
+    const int lane = threadIdx.x & 31;
+    const int64_t tiles_c = (cols + 127) >> 7;
+    const int64_t ntiles = ((rows + 127) >> 7) * tiles_c;
+    tile_pipeline<T>(&map, ntiles, tiles_c, err, [&](const uint8_t* tile, int64_t t, auto&& release) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        Block8x8<T> blk;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lds_vec8<T>(tile, 8 * group + i, strip, blk.row[i]);
+        float cm[8], rm[8];
+        blk.col_absmax(cm);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float f[8];
+            blk.row[i].get(f);
+            rm[i] = absmax8(f);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            cm[j] = fmaxf(cm[j], __shfl_xor_sync(0xffffffffu, cm[j], 8));
+            cm[j] = fmaxf(cm[j], __shfl_xor_sync(0xffffffffu, cm[j], 16));
+            rm[j] = fmaxf(rm[j], __shfl_xor_sync(0xffffffffu, rm[j], 1));
+            rm[j] = fmaxf(rm[j], __shfl_xor_sync(0xffffffffu, rm[j], 2));
+            rm[j] = fmaxf(rm[j], __shfl_xor_sync(0xffffffffu, rm[j], 4));
+        }
+        if (lane < 8) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) s_cpart[wr][8 * strip + j] = cm[j];
+        }
+        if ((lane & 7) == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s_rpart[wc][8 * group + i] = rm[i];
+        }
+        __syncthreads();
+        release();
+        // threads 0..127: one scale per tile column; 128..255: one per tile row
+        if (threadIdx.x < 128) {
+            const int c = threadIdx.x;
+            const float sc = scale_from_amax(fmaxf(fmaxf(s_cpart[0][c], s_cpart[1][c]), fmaxf(s_cpart[2][c], s_cpart[3][c])));
+            s_cscale[c] = sc;
+            const int64_t cg = (tc << 7) + c;
+            if (cg < cols) sinvt[cg + tr * ld_st] = __frcp_rn(sc);
+        } else {
+            const int r = threadIdx.x - 128;
+            const float sr = scale_from_amax(fmaxf(s_rpart[0][r], s_rpart[1][r]));
+            s_rscale[r] = sr;
+            const int64_t rg = (tr << 7) + r;
+            if (rg < rows) sinv[rg + tc * ld_s] = __frcp_rn(sr);
+        }
+        __syncthreads();
+        const int64_t r0 = (tr << 7) + 8 * group;
+        const int64_t c0 = (tc << 7) + 8 * strip;
+        if (c0 < cols && r0 < rows) {          // rows, cols % 16 == 0: 8-blocks are all-in or all-out
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float f[8];
+                blk.row[i].get(f);
+                *reinterpret_cast<uint2*>(q + (r0 + i) * ldq + c0) = quant8(f, s_rscale[8 * group + i]);
+            }
+            const float4 sa = *reinterpret_cast<const float4*>(&s_cscale[8 * strip]);
+            const float4 sb = *reinterpret_cast<const float4*>(&s_cscale[8 * strip + 4]);
+            const float sc[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint2*>(qt + (c0 + j) * ldqt + r0) = blk.quant_col(j, sc[j]);
+        }
+        __syncthreads();                       // the shared arrays are rewritten by the next tile
+    });
+}
+
 // 128x128 tiles: amax over the tile (shuffles + shared memory), then
 // row-major and/or transposed bytes straight from registers.
 template <typename T>

@@ -10,8 +10,10 @@ pytorch/ao PR #4209 (Findings So Far and review thread):
   dgrad    dx = dy . W      A = dy (1x128 along N),         B^T = W^T (128x128, same tiles)
   wgrad    dW = dy^T . x    A = dy^T (1x128 along tokens),  B^T = x^T (1x128 along tokens)
 
-x: M x K, W: N x K, dy: M x N (all bf16); outputs bf16.  Five quantization
-launches (x, x^T, W with W^T, dy, dy^T) and three GEMM launches per step.
+x: M x K, W: N x K, dy: M x N (all bf16); outputs bf16.  Three quantization
+launches per step -- x in both 1x128 directions from one read, W with its
+transposed copy, dy in both directions from one read -- and three GEMM
+launches.
 """
 from __future__ import annotations
 
@@ -23,7 +25,7 @@ from . import ops
 class Fp8LinearStep:
     """Preallocated buffers for one (M, N, K) linear layer's fwd + bwd."""
 
-    LAUNCHES_PER_STEP = 8
+    LAUNCHES_PER_STEP = 6
 
     def __init__(self, M: int, N: int, K: int, device="cuda"):
         self.M, self.N, self.K = M, N, K
@@ -50,11 +52,9 @@ class Fp8LinearStep:
         self.workspace = torch.empty((max(ws, 16),), dtype=u8, device=d)
 
     def quantize(self, x: torch.Tensor, W: torch.Tensor, dy: torch.Tensor):
-        ops.fp8_quant_1x128(x, q=self.xq, scale_inv=self.xs)
-        ops.fp8_quant_1x128(x, transpose_out=True, q=self.xtq, scale_inv=self.xts)
+        ops.fp8_quant_1x128_dual(x, out=(self.xq, self.xs, self.xtq, self.xts))
         ops.fp8_quant_128x128(W, want_q=True, want_qt=True, out=(self.wq, self.ws, self.wtq, self.wts))
-        ops.fp8_quant_1x128(dy, q=self.dyq, scale_inv=self.dys)
-        ops.fp8_quant_1x128(dy, transpose_out=True, q=self.dytq, scale_inv=self.dyts)
+        ops.fp8_quant_1x128_dual(dy, out=(self.dyq, self.dys, self.dytq, self.dyts))
 
     def gemms(self, mark=None):
         """The three GEMMs; `mark(i)` (optional) is called before GEMM i and
@@ -82,14 +82,13 @@ class Fp8LinearStep:
         return 2.0 * self.M * self.N * self.K
 
     def quant_bytes(self) -> float:
-        """Algorithmic HBM bytes of the five quantization launches: bf16 read +
-        e4m3 write per element, plus 4 bytes per scale written."""
+        """Algorithmic HBM bytes of the three quantization launches: each bf16
+        input read once (2 B per element), two e4m3 outputs written (2 x 1 B
+        per element), plus 4 bytes per scale written."""
         M, N, K = self.M, self.N, self.K
         cd = lambda a: (a + 127) // 128
         b = 0.0
-        b += M * K * 3 + 4 * M * cd(K)            # x 1x128
-        b += M * K * 3 + 4 * K * cd(M)            # x^T along tokens
-        b += N * K * 4 + 2 * 4 * cd(N) * cd(K)    # W 128x128 + transposed copy (2 B in, 2 x 1 B out)
-        b += M * N * 3 + 4 * M * cd(N)            # dy 1x128
-        b += M * N * 3 + 4 * N * cd(M)            # dy^T along tokens
+        b += M * K * 4 + 4 * M * cd(K) + 4 * K * cd(M)     # x: 1x128 along K and along tokens
+        b += N * K * 4 + 2 * 4 * cd(N) * cd(K)             # W 128x128 + transposed copy
+        b += M * N * 4 + 4 * M * cd(N) + 4 * N * cd(M)     # dy: 1x128 along N and along tokens
         return b

@@ -49,6 +49,7 @@ def lib():
         L = ctypes.CDLL(path)
         p, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
         L.fp8_quant_1x128.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, i32, p]
+        L.fp8_quant_1x128_dual.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, p, i64, p, i64, p]
         L.fp8_quant_128x128.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, p, i64, p, i64, p]
         L.fp8_quant_tensor_workspace_size.argtypes = [i64]
         L.fp8_quant_tensor_workspace_size.restype = sz
@@ -60,8 +61,8 @@ def lib():
         L.fp8bs_status_string.argtypes = [i32]
         L.fp8bs_status_string.restype = ctypes.c_char_p
         L.fp8bs_check_device_error.argtypes = [p]
-        for fn in ("fp8_quant_1x128", "fp8_quant_128x128", "fp8_quant_tensor", "fp8_quant_rowwise",
-                   "fp8_scaled_gemm", "fp8bs_check_device_error"):
+        for fn in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_tensor",
+                   "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8bs_check_device_error"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -127,6 +128,27 @@ def fp8_quant_1x128(x: torch.Tensor, transpose_out: bool = False, q: Optional[to
     _check("fp8_quant_1x128", lib().fp8_quant_1x128(x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(), q.stride(0),
                                                     s.data_ptr(), ld_s, int(transpose_out), _stream(x)))
     return q, s
+
+
+def fp8_quant_1x128_dual(x: torch.Tensor, out=None):
+    """Both 1x128 quantizations from one read of x: returns (q, scale_inv,
+    q_t, scale_inv_t), equal to fp8_quant_1x128(x) followed by
+    fp8_quant_1x128(x, transpose_out=True).  Preallocated outputs may be
+    passed as out=(q, scale_inv, q_t, scale_inv_t)."""
+    rows, cols = x.shape
+    xt = _dtype_code(x)
+    if out is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+        s = colmajor_grid(rows, (cols + 127) // 128, x.device)
+        qt = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+        st = colmajor_grid(cols, (rows + 127) // 128, x.device)
+    else:
+        q, s, qt, st = out
+    _check("fp8_quant_1x128_dual",
+           lib().fp8_quant_1x128_dual(x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(), q.stride(0), s.data_ptr(),
+                                      _grid_ld(s, rows), qt.data_ptr(), qt.stride(0), st.data_ptr(), _grid_ld(st, cols),
+                                      _stream(x)))
+    return q, s, qt, st
 
 
 def fp8_quant_128x128(x: torch.Tensor, want_q: bool = True, want_qt: bool = False, out=None):

@@ -10,6 +10,7 @@ only the named kernel runs R times):
   gemm_longk   256 x 512 x 128128 (k_blocks 1001), 1x128 x 128x128, split-K, bf16 out
   quant_rows   1x128 quantization of a 32768 x 32768 bf16 matrix
   quant_cols   1x128 along rows (transposed output) of a 16640 x 8192 bf16 matrix
+  quant_dual   both 1x128 directions from one read of a 16640 x 8192 bf16 matrix
   quant_tile   128x128 quantization (with transposed copy) of a 32768 x 32768 bf16 matrix
 With --time, each launch is timed with CUDA events and the mean is printed.
 """
@@ -64,6 +65,11 @@ def _quant_case(name):
         q, s = ops.fp8_quant_1x128(x, transpose_out=True)
         nbytes = x.numel() * 3 + 4 * s.numel()
         fn = lambda: ops.fp8_quant_1x128(x, transpose_out=True, q=q, scale_inv=s)
+    elif name == "quant_dual":
+        x = inputs.llama4(5120, 8192)[0].cuda()
+        out = ops.fp8_quant_1x128_dual(x)
+        nbytes = x.numel() * 4 + 4 * (out[1].numel() + out[3].numel())
+        fn = lambda: ops.fp8_quant_1x128_dual(x, out=out)
     else:
         x = inputs.quant_sweep(32768).cuda()
         if name == "quant_rows":

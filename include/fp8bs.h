@@ -93,6 +93,40 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
                              int transpose_out, cudaStream_t stream);
 
 /*
+ * fp8_quant_1x128_dual -- both 1x128 quantizations of one tensor from a
+ * single read of it.
+ *
+ * Defined by: the two operand recipes of the FP8 blockwise linear layer in
+ * pytorch/ao PR #2785 "integrate torch._scaled_mm into Float8BlockwiseLinear
+ * and add bench script" (Summary): the activation is quantized 1x128 along
+ * its contiguous dimension for the forward GEMM and 1x128 along tokens (the
+ * rows) for the weight-gradient GEMM; likewise the output gradient for the
+ * input-gradient and weight-gradient GEMMs.  The group rule is that of
+ * fp8_quant_1x128 (pytorch/ao PR #2592, block shape (1,128)).
+ *
+ * The results are byte-identical to the two calls
+ *     fp8_quant_1x128(x, ..., q,   ldq,   scale_inv,   ld_scale,   0, stream)
+ *     fp8_quant_1x128(x, ..., q_t, ldq_t, scale_inv_t, ld_scale_t, 1, stream)
+ * with the layouts documented there:
+ *     q:           rows x cols, leading dim ldq >= cols;
+ *     scale_inv:   scale_inv[r + g*ld_scale], g < ceil(cols/128), ld_scale >= rows;
+ *     q_t:         cols x rows (the transpose), leading dim ldq_t >= rows;
+ *     scale_inv_t: scale_inv_t[c + g*ld_scale_t], g < ceil(rows/128), ld_scale_t >= cols.
+ * All four outputs are written; none may be null and none may overlap x or
+ * one another.  The caller owns every buffer.
+ * Alignment: x and the four outputs 16-byte aligned; ldx*sizeof(xt), ldq and
+ * ldq_t multiples of 16 bytes; rows % 16 == 0 and cols % 16 == 0; ld_scale and
+ * ld_scale_t % 4 == 0.  Otherwise FP8BS_ERR_ALIGNMENT.  Other argument errors:
+ * FP8BS_ERR_INVALID_ARG (null pointer, size < 1, leading dimension too small),
+ * FP8BS_ERR_UNSUPPORTED (unknown dtype).  Nothing is launched when a check
+ * fails.  Asynchronous on `stream`.
+ */
+fp8bs_status fp8_quant_1x128_dual(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                                  uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale,
+                                  uint8_t* q_t, int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t,
+                                  cudaStream_t stream);
+
+/*
  * fp8_quant_128x128 -- dynamic quantization with one scale per 128x128 tile.
  *
  * Defined by: pytorch/ao PR #2592 (Performance table, block shape (128,128));

@@ -32,8 +32,8 @@ def L():
 
 def test_header_declares_the_path(L):
     names = declared_functions()
-    for want in ("fp8_quant_1x128", "fp8_quant_128x128", "fp8_quant_tensor", "fp8_quant_rowwise",
-                 "fp8_scaled_gemm", "fp8_scaled_gemm_workspace_size", "fp8bs_status_string",
+    for want in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_tensor",
+                 "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_workspace_size", "fp8bs_status_string",
                  "fp8bs_check_device_error", "fp8_quant_tensor_workspace_size"):
         assert want in names
 
@@ -64,6 +64,30 @@ def test_quant_1x128_validation(L):
     assert q1x128(L, ldq=260) == ALIGN
     assert q1x128(L, lds=258) == ALIGN
     assert q1x128(L, rows=200, lds=256, t=1) == ALIGN         # transposed needs rows % 16
+
+
+def qdual(L, x=GOOD, xt=0, rows=256, cols=384, ldx=384, q=GOOD, ldq=384, s=GOOD, lds=256, qt=GOOD, ldqt=256,
+          st=GOOD, ldst=384):
+    return L.fp8_quant_1x128_dual(x, xt, rows, cols, ldx, q, ldq, s, lds, qt, ldqt, st, ldst, None)
+
+
+def test_quant_1x128_dual_validation(L):
+    for kw in ({"x": 0}, {"q": 0}, {"s": 0}, {"qt": 0}, {"st": 0}, {"rows": 0}, {"cols": 0}):
+        assert qdual(L, **kw) == INVALID, kw
+    assert qdual(L, ldx=256) == INVALID              # ldx < cols
+    assert qdual(L, ldq=368) == INVALID              # ldq < cols
+    assert qdual(L, lds=240) == INVALID              # ld_scale < rows
+    assert qdual(L, ldqt=240) == INVALID             # ldq_t < rows
+    assert qdual(L, ldst=368) == INVALID             # ld_scale_t < cols
+    assert qdual(L, xt=5) == UNSUPPORTED
+    for kw in ({"x": BAD}, {"q": BAD}, {"s": BAD}, {"qt": BAD}, {"st": BAD}):
+        assert qdual(L, **kw) == ALIGN, kw
+    assert qdual(L, rows=200, lds=200, ldqt=208) == ALIGN       # rows % 16
+    assert qdual(L, cols=200, ldx=200, ldq=208, ldst=200) == ALIGN   # cols % 16
+    assert qdual(L, ldq=392) == ALIGN                # ldq % 16
+    assert qdual(L, ldqt=264) == ALIGN               # ldq_t % 16
+    assert qdual(L, lds=258) == ALIGN                # ld_scale % 4
+    assert qdual(L, ldx=388) == ALIGN                # bf16 rows of 776 bytes: not a multiple of 16
 
 
 def test_quant_128x128_validation(L):

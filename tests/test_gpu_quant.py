@@ -52,6 +52,70 @@ def test_quant_1x128_transposed(R, C, dt):
     check_1x128(inputs.random_matrix(R, C, seed=R * 3 + C, dtype=dt), transpose=True)
 
 
+def check_dual(x_cpu):
+    """fp8_quant_1x128_dual against the oracle's two 1x128 directions, and
+    against the two single-direction launches, byte for byte."""
+    xd = dev(x_cpu)
+    q, s, qt, st = ops.fp8_quant_1x128_dual(xd)
+    q1, s1 = ops.fp8_quant_1x128(xd)
+    qt1, st1 = ops.fp8_quant_1x128(xd, transpose_out=True)
+    torch.cuda.synchronize()
+    xb = bits(x_cpu)
+    qo, so = oracle.quant_1x128(xb)
+    assert_bytes_equal(q, qo, "q")
+    assert_scales_equal(grid_np(s), so, "scale_inv")
+    qto, sto = oracle.quant_1x128(xb, transpose=True)
+    assert_bytes_equal(qt, qto, "q_t")
+    assert_scales_equal(grid_np(st), sto, "scale_inv_t")
+    assert torch.equal(q, q1) and torch.equal(qt, qt1)
+    assert_scales_equal(grid_np(s), grid_np(s1), "scale_inv vs single-direction launch")
+    assert_scales_equal(grid_np(st), grid_np(st1), "scale_inv_t vs single-direction launch")
+
+
+@pytest.mark.parametrize("R,C,dt", [(304, 400, torch.bfloat16), (256, 1024, torch.float32), (16, 16, torch.bfloat16),
+                                    (1040, 272, torch.bfloat16), (128, 130 * 16, torch.float32),
+                                    (400, 144, torch.float32), (2048, 1024, torch.bfloat16)])
+def test_quant_1x128_dual(R, C, dt):
+    """Both directions from one read: several tiles, ragged last tile row and
+    column (sizes multiples of 16, not of 128), both input dtypes."""
+    check_dual(inputs.random_matrix(R, C, seed=R * 5 + C, dtype=dt))
+
+
+def test_quant_1x128_dual_special_values():
+    """Groups whose row and column maxima differ by orders of magnitude inside
+    one tile (zeros, +-0, 448 exactly, near-fp32-max, subnormal-range values),
+    so that a row scale used for a column group (or the reverse) shows."""
+    x = inputs.random_matrix(256, 384, seed=9, dtype=torch.float32)
+    x[0, :128] = 0.0
+    x[1, :128] = -0.0
+    x[:, 5] = 0.0
+    x[2, :] = 448.0
+    x[:, 200] = 3.0e38
+    x[3, 130:250] = 1e-30
+    x[130:140, 300:310] = -2.0 ** -9
+    check_dual(x)
+
+
+def test_quant_1x128_dual_full_size_sampled():
+    """The Llama4 activation (16640 x 8192 bf16) in the launch the linear
+    step uses; sampled rows of the row direction and sampled rows of the
+    transposed direction against the oracle."""
+    x = inputs.llama4(5120, 8192)[0]
+    xd = dev(x)
+    q, s, qt, st = ops.fp8_quant_1x128_dual(xd)
+    torch.cuda.synchronize()
+    xb = bits(x)
+    M, K = x.shape
+    rows = [0, 1, 127, 128, M // 2 + 3, M - 1]
+    qo, so = oracle.quant_1x128(xb, rows=rows)
+    assert_bytes_equal(q[torch.as_tensor(rows, device="cuda")], qo, "q (sampled rows)")
+    assert_scales_equal(grid_np(s)[rows], so, "scale_inv (sampled rows)")
+    cols = [0, 5, 128, K // 2 + 1, K - 1]
+    qto, sto = oracle.quant_1x128(xb, transpose=True, rows=cols)
+    assert_bytes_equal(qt[torch.as_tensor(cols, device="cuda")], qto, "q_t (sampled rows)")
+    assert_scales_equal(grid_np(st)[cols], sto, "scale_inv_t (sampled rows)")
+
+
 @pytest.mark.parametrize("R,C,dt", [(304, 400, torch.bfloat16), (1024, 512, torch.float32), (16, 16, torch.bfloat16),
                                     (128, 128, torch.float32), (384, 1040, torch.bfloat16)])
 def test_quant_128x128_with_transpose(R, C, dt):
