@@ -174,6 +174,14 @@ fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap
     if (!d->gemm_attr_set[MODE]) {
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::alloc) != cudaSuccess)
             return FP8BS_ERR_CUDA;
+        if (EpiCfg<MODE>::reg_split) {
+            // the warpgroups' register hand-over is sized for this exact
+            // allocation at launch; with fewer registers the promotion warps'
+            // increase could never be granted, so refuse to launch instead
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return FP8BS_ERR_CUDA;
+            if (fa.numRegs != EpiCfg<MODE>::launch_regs) return FP8BS_ERR_UNSUPPORTED;
+        }
         d->gemm_attr_set[MODE] = true;
     }
     const int grid = (int)std::min<int64_t>(p.num_units, d->num_sms);

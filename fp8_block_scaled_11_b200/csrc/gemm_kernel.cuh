@@ -18,7 +18,9 @@
 //               TMEM accumulators and commits the accumulator and the smem
 //               stage when the MMAs complete.
 //   warps 2..   promotion / epilogue (8 warps, or 16 for the 1x128 x 1x128
-//               recipe whose per-column scales double the per-element work):
+//               recipe whose per-column scales double the per-element work;
+//               those 16 are warps 4..19, after a first warpgroup whose two
+//               idle warps let it hand its registers over to them):
 //               per accumulation group (one K-block for the block recipes; the
 //               whole K range for tensor/rowwise) they tcgen05.ld the partial
 //               sums, multiply by the scale product and add into fp32 registers
@@ -71,16 +73,37 @@ struct SmemLayout {
 
 enum GemmMode : int { kModeTensor = 0, kModeRowwise = 1, kModeBlock128 = 2, kModeBlock1x128 = 3 };
 
-// Promotion-warp configuration per recipe (measured on B200: the 1x128 x
-// 128x128 recipe is fastest with 8 warps loading one 16-column TMEM chunk at a
-// time, the 1x128 x 1x128 recipe with 16 warps keeping two chunks in flight).
+// Warp roles per recipe.  Warp 0 issues the TMA loads, warp 1 the MMAs, the
+// rest promote and store.  With `reg_split` the first warpgroup (producer, MMA
+// issuer and two idle warps) hands registers over to the promotion warps
+// (setmaxnreg), which then run their loop without spills; the hand-over is
+// sized for exactly `launch_regs` registers per thread at launch, which the
+// host checks before the first launch.  Measured on B200: the 1x128 x 128x128
+// recipe is fastest with 8 promotion warps loading one 16-column TMEM chunk at
+// a time (168 registers, no hand-over needed), the 1x128 x 1x128 recipe with
+// 16 promotion warps keeping two chunks in flight, at 104 registers after the
+// hand-over (96 at launch, where the loop spilled: 6% slower).
 template <int MODE>
 struct EpiCfg {
     static constexpr int warps = MODE == kModeBlock1x128 ? 16 : 8;
+    static constexpr bool reg_split = MODE == kModeBlock1x128;
     static constexpr bool single_buf = MODE == kModeBlock128;
-    static constexpr int threads = 64 + 32 * warps;
+    static constexpr int ctrl_warps = reg_split ? 4 : 2;
+    static constexpr int threads = 32 * (ctrl_warps + warps);
     static constexpr int cols = kBN * 4 / warps;        // accumulator columns per thread
     static constexpr int chunks = cols / 16;            // 16-column TMEM loads per group
+    // registers per thread at launch: the per-sub-partition limit of
+    // __launch_bounds__(threads, 1) (16384 registers shared by the
+    // ceil(warps / 4) warps of each SM sub-partition, in steps of 8); after
+    // the hand-over the first warpgroup keeps ctrl_regs, the promotion warps
+    // take the rest (at most 232)
+    static constexpr int launch_regs = (16384 / (32 * ((ctrl_warps + warps + 3) / 4))) / 8 * 8;
+    static constexpr int ctrl_regs = 40;
+    static constexpr int epi_regs_raw = (threads * launch_regs - 128 * ctrl_regs) / (32 * warps) / 8 * 8;
+    static constexpr int epi_regs = epi_regs_raw > 232 ? 232 : epi_regs_raw;
+    static_assert(!reg_split || (ctrl_warps == 4 && warps % 4 == 0 &&
+                                 128 * ctrl_regs + 32 * warps * epi_regs <= threads * launch_regs),
+                  "register hand-over exceeds the launch allocation");
 };
 
 struct GemmParams {
@@ -193,112 +216,117 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         atomicOr(p.err, 1);
     };
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int ss = 0;
-            uint32_t sphase = 0;
-            bool ok = true;
-            // per stage: was it ever filled, and the parity of its latest fill
-            uint32_t filled = 0, fill_par = 0, sfilled = 0, sfill_par = 0;
-            auto issue_scales = [&](int m0, int n0, int kb) -> bool {
-                if (!mbar_wait_bounded(sc_empty(ss), sphase ^ 1u, abort_flag, kWaitLimitNs)) return false;
-                const uint32_t dst = sbase + SmemLayout::sc_off + ss * kScaleEntryBytes;
-                mbar_arrive_expect_tx(sc_full(ss), kScaleTx);
-                tma_load_2d(dst, &tmSA, sc_full(ss), m0, kb);
-                if (kColScales) {
-                    tma_load_2d(dst + kBM * 4, &tmSB, sc_full(ss), n0, kb);
-                } else {
-                    tma_load_2d(dst + kBM * 4, &tmSB, sc_full(ss), (n0 / 128) & ~3, kb);
-                }
-                sfilled |= 1u << ss;
-                sfill_par = (sfill_par & ~(1u << ss)) | (sphase << ss);
-                if (++ss == kScaleStages) { ss = 0; sphase ^= 1u; }
-                return true;
-            };
-            for (int64_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-                int tm, tn, kb0, kb1, split;
-                decode_unit(p, u, tm, tn, kb0, kb1, split);
-                const int m0 = tm * kBM, n0 = tn * kBN;
-                if (MODE == kModeRowwise) ok = issue_scales(m0, n0, 0);
-                for (int kb = kb0; kb < kb1 && ok; ++kb) {
-                    if (!mbar_wait_bounded(ab_empty(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-                    mbar_arrive_expect_tx(ab_full(stage), kATileBytes + kBTileBytes);
-                    tma_load_2d(sbase + SmemLayout::a_off + stage * kATileBytes, &tmA, ab_full(stage), kb * kBK, m0);
-                    tma_load_2d(sbase + SmemLayout::b_off + stage * kBTileBytes, &tmB, ab_full(stage), kb * kBK, n0);
-                    filled |= 1u << stage;
-                    fill_par = (fill_par & ~(1u << stage)) | (phase << stage);
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
-                    if (kPromote && kScaleRing) ok = issue_scales(m0, n0, kb);
-                }
-            }
-            if (!ok) give_up();
-            // drain: every issued TMA copy must have landed before the CTA exits
-            for (int s = 0; s < kStages; ++s)
-                if (filled >> s & 1u) mbar_wait_bounded(ab_full(s), fill_par >> s & 1u, nullptr, kDrainLimitNs);
-            for (int s = 0; s < kScaleStages; ++s)
-                if (sfilled >> s & 1u) mbar_wait_bounded(sc_full(s), sfill_par >> s & 1u, nullptr, kDrainLimitNs);
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_e4m3_f32(kBM, kBN);
-            int stage = 0;
-            uint32_t phase = 0;
-            int tb = 0;
-            uint32_t tphase = 0;
-            bool ok = true, issued = false;
-            for (int64_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-                int tm, tn, kb0, kb1, split;
-                decode_unit(p, u, tm, tn, kb0, kb1, split);
-                const int ngroups = kPromote ? (kb1 - kb0) : 1;
-                int kb = kb0;
-                for (int g = 0; g < ngroups && ok; ++g) {
-                    const int kb_end = kPromote ? kb + 1 : kb1;
-                    // The smem stage of the group's first K-block is normally
-                    // ready long before the TMEM buffer is free: wait for it
-                    // first, so that only the TMEM hand-off is on the critical path.
-                    if (!mbar_wait_bounded(ab_full(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-                    if (!mbar_wait_bounded(tm_empty(tb), tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + (uint32_t)(tb * kBN);
-                    const int kb_first = kb;         // its stage was waited for above
-                    for (; kb < kb_end; ++kb) {
-                        if (kb != kb_first) {
-                            if (!mbar_wait_bounded(ab_full(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-                            tc_fence_after();
-                        }
-                        const uint32_t a_addr = sbase + SmemLayout::a_off + stage * kATileBytes;
-                        const uint32_t b_addr = sbase + SmemLayout::b_off + stage * kBTileBytes;
-#pragma unroll
-                        for (int k = 0; k < kBK / 32; ++k) {
-                            const uint64_t adesc = smem_desc_k_sw128(a_addr + k * 32);
-                            const uint64_t bdesc = smem_desc_k_sw128(b_addr + k * 32);
-                            const uint32_t acc = (kPromote ? (k > 0) : (kb > kb0 || k > 0)) ? 1u : 0u;
-                            umma_f8(d_tmem, adesc, bdesc, idesc, acc);
-                        }
-                        issued = true;
-                        // the accumulator hand-off is on the critical path: signal it first
-                        if (kb + 1 == kb_end) umma_commit(tm_full(tb));
-                        umma_commit(ab_empty(stage));
-                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+    if (warp < E::ctrl_warps) {
+        // the first warpgroup's roles (its hand-over is warpgroup-uniform)
+        if constexpr (E::reg_split) setmaxnreg_dec<E::ctrl_regs>();
+        if (warp == 0) {
+            // ------------------------------------------------------------ producer
+            if (lane == 0) {
+                int stage = 0;
+                uint32_t phase = 0;
+                int ss = 0;
+                uint32_t sphase = 0;
+                bool ok = true;
+                // per stage: was it ever filled, and the parity of its latest fill
+                uint32_t filled = 0, fill_par = 0, sfilled = 0, sfill_par = 0;
+                auto issue_scales = [&](int m0, int n0, int kb) -> bool {
+                    if (!mbar_wait_bounded(sc_empty(ss), sphase ^ 1u, abort_flag, kWaitLimitNs)) return false;
+                    const uint32_t dst = sbase + SmemLayout::sc_off + ss * kScaleEntryBytes;
+                    mbar_arrive_expect_tx(sc_full(ss), kScaleTx);
+                    tma_load_2d(dst, &tmSA, sc_full(ss), m0, kb);
+                    if (kColScales) {
+                        tma_load_2d(dst + kBM * 4, &tmSB, sc_full(ss), n0, kb);
+                    } else {
+                        tma_load_2d(dst + kBM * 4, &tmSB, sc_full(ss), (n0 / 128) & ~3, kb);
                     }
-                    if (!ok) break;
-                    if (++tb == kTmemBufs) { tb = 0; tphase ^= 1u; }
+                    sfilled |= 1u << ss;
+                    sfill_par = (sfill_par & ~(1u << ss)) | (sphase << ss);
+                    if (++ss == kScaleStages) { ss = 0; sphase ^= 1u; }
+                    return true;
+                };
+                for (int64_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                    int tm, tn, kb0, kb1, split;
+                    decode_unit(p, u, tm, tn, kb0, kb1, split);
+                    const int m0 = tm * kBM, n0 = tn * kBN;
+                    if (MODE == kModeRowwise) ok = issue_scales(m0, n0, 0);
+                    for (int kb = kb0; kb < kb1 && ok; ++kb) {
+                        if (!mbar_wait_bounded(ab_empty(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                        mbar_arrive_expect_tx(ab_full(stage), kATileBytes + kBTileBytes);
+                        tma_load_2d(sbase + SmemLayout::a_off + stage * kATileBytes, &tmA, ab_full(stage), kb * kBK, m0);
+                        tma_load_2d(sbase + SmemLayout::b_off + stage * kBTileBytes, &tmB, ab_full(stage), kb * kBK, n0);
+                        filled |= 1u << stage;
+                        fill_par = (fill_par & ~(1u << stage)) | (phase << stage);
+                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                        if (kPromote && kScaleRing) ok = issue_scales(m0, n0, kb);
+                    }
                 }
+                if (!ok) give_up();
+                // drain: every issued TMA copy must have landed before the CTA exits
+                for (int s = 0; s < kStages; ++s)
+                    if (filled >> s & 1u) mbar_wait_bounded(ab_full(s), fill_par >> s & 1u, nullptr, kDrainLimitNs);
+                for (int s = 0; s < kScaleStages; ++s)
+                    if (sfilled >> s & 1u) mbar_wait_bounded(sc_full(s), sfill_par >> s & 1u, nullptr, kDrainLimitNs);
             }
-            if (!ok) give_up();
-            if (issued) {
-                // all MMAs of this thread complete before TMEM can be freed
-                umma_commit(drain_bar);
-                mbar_wait_bounded(drain_bar, 0, nullptr, kDrainLimitNs);
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc = idesc_e4m3_f32(kBM, kBN);
+                int stage = 0;
+                uint32_t phase = 0;
+                int tb = 0;
+                uint32_t tphase = 0;
+                bool ok = true, issued = false;
+                for (int64_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                    int tm, tn, kb0, kb1, split;
+                    decode_unit(p, u, tm, tn, kb0, kb1, split);
+                    const int ngroups = kPromote ? (kb1 - kb0) : 1;
+                    int kb = kb0;
+                    for (int g = 0; g < ngroups && ok; ++g) {
+                        const int kb_end = kPromote ? kb + 1 : kb1;
+                        // The smem stage of the group's first K-block is normally
+                        // ready long before the TMEM buffer is free: wait for it
+                        // first, so that only the TMEM hand-off is on the critical path.
+                        if (!mbar_wait_bounded(ab_full(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                        if (!mbar_wait_bounded(tm_empty(tb), tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t d_tmem = tmem_base + (uint32_t)(tb * kBN);
+                        const int kb_first = kb;         // its stage was waited for above
+                        for (; kb < kb_end; ++kb) {
+                            if (kb != kb_first) {
+                                if (!mbar_wait_bounded(ab_full(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                                tc_fence_after();
+                            }
+                            const uint32_t a_addr = sbase + SmemLayout::a_off + stage * kATileBytes;
+                            const uint32_t b_addr = sbase + SmemLayout::b_off + stage * kBTileBytes;
+    #pragma unroll
+                            for (int k = 0; k < kBK / 32; ++k) {
+                                const uint64_t adesc = smem_desc_k_sw128(a_addr + k * 32);
+                                const uint64_t bdesc = smem_desc_k_sw128(b_addr + k * 32);
+                                const uint32_t acc = (kPromote ? (k > 0) : (kb > kb0 || k > 0)) ? 1u : 0u;
+                                umma_f8(d_tmem, adesc, bdesc, idesc, acc);
+                            }
+                            issued = true;
+                            // the accumulator hand-off is on the critical path: signal it first
+                            if (kb + 1 == kb_end) umma_commit(tm_full(tb));
+                            umma_commit(ab_empty(stage));
+                            if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                        }
+                        if (!ok) break;
+                        if (++tb == kTmemBufs) { tb = 0; tphase ^= 1u; }
+                    }
+                }
+                if (!ok) give_up();
+                if (issued) {
+                    // all MMAs of this thread complete before TMEM can be freed
+                    umma_commit(drain_bar);
+                    mbar_wait_bounded(drain_bar, 0, nullptr, kDrainLimitNs);
+                }
             }
         }
     } else {
+        if constexpr (E::reg_split) setmaxnreg_inc<E::epi_regs>();
         // ------------------------------------------------------------ promotion / epilogue
-        const int e = warp - 2;                 // 0 .. kEpiWarps-1
+        const int e = warp - E::ctrl_warps;     // 0 .. kEpiWarps-1
         const int lq = warp & 3;                // TMEM lane quarter this warp may access
         const int col0 = (e >> 2) * kColsPerThread;   // this warp's columns within the tile
         const int row_in_tile = lq * 32 + lane;

@@ -189,6 +189,21 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16])
                  : "memory");
 }
 
+// Warpgroup register hand-over: every warp of the warpgroup executes the same
+// instruction.  A decrease returns registers to the CTA's pool; an increase
+// waits until the pool holds enough, so the increases of a kernel must never
+// ask for more than the decreases and the launch leave free.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // 16-byte shared-memory load that stays in program order with the
 // surrounding volatile asm (keeps the scale vector from being hoisted).
 __device__ __forceinline__ float4 lds128(uint32_t addr)
