@@ -19,8 +19,9 @@
 //               stage when the MMAs complete.
 //   warps 2..   promotion / epilogue (8 warps, or 16 for the 1x128 x 1x128
 //               recipe whose per-column scales double the per-element work;
-//               those 16 are warps 4..19, after a first warpgroup whose two
-//               idle warps let it hand its registers over to them):
+//               with both block recipes the promotion warps start at warp 4,
+//               after a first warpgroup whose two idle warps let it hand its
+//               registers over to them):
 //               per accumulation group (one K-block for the block recipes; the
 //               whole K range for tensor/rowwise) they tcgen05.ld the partial
 //               sums, multiply by the scale product and add into fp32 registers
@@ -79,14 +80,15 @@ enum GemmMode : int { kModeTensor = 0, kModeRowwise = 1, kModeBlock128 = 2, kMod
 // (setmaxnreg), which then run their loop without spills; the hand-over is
 // sized for exactly `launch_regs` registers per thread at launch, which the
 // host checks before the first launch.  Measured on B200: the 1x128 x 128x128
-// recipe is fastest with 8 promotion warps loading one 16-column TMEM chunk at
-// a time (168 registers, no hand-over needed), the 1x128 x 1x128 recipe with
+// recipe is fastest with 8 promotion warps at 232 registers that issue four
+// 16-column TMEM loads per wait (the per-warp promotion time follows the
+// number of load round trips, not the bytes), the 1x128 x 1x128 recipe with
 // 16 promotion warps keeping two chunks in flight, at 104 registers after the
 // hand-over (96 at launch, where the loop spilled: 6% slower).
 template <int MODE>
 struct EpiCfg {
     static constexpr int warps = MODE == kModeBlock1x128 ? 16 : 8;
-    static constexpr bool reg_split = MODE == kModeBlock1x128;
+    static constexpr bool reg_split = MODE == kModeBlock1x128 || MODE == kModeBlock128;
     static constexpr bool single_buf = MODE == kModeBlock128;
     static constexpr int ctrl_warps = reg_split ? 4 : 2;
     static constexpr int threads = 32 * (ctrl_warps + warps);
@@ -104,6 +106,7 @@ struct EpiCfg {
     static_assert(!reg_split || (ctrl_warps == 4 && warps % 4 == 0 &&
                                  128 * ctrl_regs + 32 * warps * epi_regs <= threads * launch_regs),
                   "register hand-over exceeds the launch allocation");
+    static_assert(!single_buf || chunks % 4 == 0, "four TMEM loads per wait");
 };
 
 struct GemmParams {
@@ -405,14 +408,22 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     }
                 };
                 if constexpr (E::single_buf) {
-                    // one 16-column load at a time; the sibling warps of the
-                    // SM sub-partition cover its latency
+                    // four 16-column loads per wait (64 registers in flight)
 #pragma unroll
-                    for (int c = 0; c < kChunks; ++c) {
-                        uint32_t r[16];
-                        tmem_ld_32x32b_x16(tcol + c * 16, r);
-                        tmem_ld_wait(r);
-                        promote(c, r);
+                    for (int h = 0; h < kChunks / 4; ++h) {
+                        uint32_t r0[16], r1[16], r2[16], r3[16];
+                        tmem_ld_32x32b_x16(tcol + (4 * h + 0) * 16, r0);
+                        tmem_ld_32x32b_x16(tcol + (4 * h + 1) * 16, r1);
+                        tmem_ld_32x32b_x16(tcol + (4 * h + 2) * 16, r2);
+                        tmem_ld_32x32b_x16(tcol + (4 * h + 3) * 16, r3);
+                        tmem_ld_wait(r0);
+                        reg_after_wait(r1);
+                        reg_after_wait(r2);
+                        reg_after_wait(r3);
+                        promote(4 * h + 0, r0);
+                        promote(4 * h + 1, r1);
+                        promote(4 * h + 2, r2);
+                        promote(4 * h + 3, r3);
                     }
                 } else {
                     // two 16-column loads in flight: chunk c+1 loads while c is promoted

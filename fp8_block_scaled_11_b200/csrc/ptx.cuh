@@ -189,6 +189,17 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16])
                  : "memory");
 }
 
+// Orders every later use of r after a preceding tcgen05.wait::ld: both are
+// volatile asm, so they keep their order, and r is an in/out operand here.
+// Used for the destination registers of loads whose wait threads only one
+// of them through.
+__device__ __forceinline__ void reg_after_wait(uint32_t (&r)[16])
+{
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
+
 // Warpgroup register hand-over: every warp of the warpgroup executes the same
 // instruction.  A decrease returns registers to the CTA's pool; an increase
 // waits until the pool holds enough, so the increases of a kernel must never
