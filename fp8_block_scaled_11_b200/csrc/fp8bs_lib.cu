@@ -15,6 +15,7 @@
 #include "fp8bs.h"
 #include "quant_kernels.cuh"
 #include "gemm_kernel.cuh"
+#include "splitk_reduce.cuh"
 
 using namespace fp8bs;
 
@@ -512,8 +513,10 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
     if (st != FP8BS_OK) return st;
     if (plan.splits > 1) {
         const int64_t chunks = M * ((N + 3) / 4);
-        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(chunks, 256), (int64_t)d->num_sms * 8));
-        splitk_reduce_kernel<<<grid, 256, 0, stream>>>(p.ws, plan.splits, M, N, plan.ldw, D, ldd, p.out_f32, vec_out);
+        const int grid = (int)std::max<int64_t>(
+            1, std::min<int64_t>(cdiv(chunks, kReduceThreads), (int64_t)d->num_sms * 16));
+        splitk_reduce_kernel<<<grid, kReduceThreads, 0, stream>>>(p.ws, plan.splits, M, N, plan.ldw, D, ldd,
+                                                                  p.out_f32, vec_out);
         st = launch_status();
     }
     return st;

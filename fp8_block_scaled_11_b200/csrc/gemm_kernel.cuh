@@ -511,40 +511,4 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
-// Split-K reduction: D[m,n] = sum over splits (fixed order) of ws[s][m][n].
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ ws, int splits, int64_t M,
-                                                            int64_t N, int64_t ldw, void* __restrict__ D,
-                                                            int64_t ldd, int out_f32, int vec_out)
-{
-    const int64_t nq = (N + 3) >> 2;          // 4-column chunks per row
-    const int64_t total = M * nq;
-    const int64_t plane = M * ldw;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = i / nq;
-        const int64_t n = (i - m * nq) << 2;
-        const float* src = ws + m * ldw + n;
-        float4 s = *reinterpret_cast<const float4*>(src);
-        for (int k = 1; k < splits; ++k) {
-            const float4 v = *reinterpret_cast<const float4*>(src + k * plane);
-            s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-        }
-        const float v[4] = {s.x, s.y, s.z, s.w};
-        if (out_f32) {
-            float* d = reinterpret_cast<float*>(D) + m * ldd + n;
-            if (vec_out && n + 4 <= N) *reinterpret_cast<float4*>(d) = s;
-            else for (int t = 0; t < (int)((N - n) < 4 ? (N - n) : 4); ++t) d[t] = v[t];
-        } else {
-            __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(D) + m * ldd + n;
-            const uint32_t lo = cvt_bf16x2(s.x, s.y), hi = cvt_bf16x2(s.z, s.w);
-            if (vec_out && n + 4 <= N) {
-                *reinterpret_cast<uint2*>(d) = make_uint2(lo, hi);
-            } else {
-                const uint32_t ww[2] = {lo, hi};
-                uint16_t* d16 = reinterpret_cast<uint16_t*>(d);
-                for (int t = 0; t < (int)((N - n) < 4 ? (N - n) : 4); ++t) d16[t] = (uint16_t)((ww[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
-            }
-        }
-    }
-}
-
 }  // namespace fp8bs
