@@ -179,18 +179,29 @@ struct QTile {
 template <typename T>
 __device__ __forceinline__ void lds_vec8(const uint8_t* tile, int r, int s, Vec8<T>& v);
 
+// 16 bytes from shared memory as an explicit shared-space load (the tile
+// pointer reaches the callers through a lambda, where a plain dereference may
+// compile to a generic load).
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
 template <>
 __device__ __forceinline__ void lds_vec8<__nv_bfloat16>(const uint8_t* tile, int r, int s, Vec8<__nv_bfloat16>& v)
 {
-    v.raw = *reinterpret_cast<const uint4*>(tile + r * QTile<__nv_bfloat16>::row_bytes + s * 16);
+    v.raw = lds_u4(smem_u32(tile) + r * QTile<__nv_bfloat16>::row_bytes + s * 16);
 }
 
 template <>
 __device__ __forceinline__ void lds_vec8<float>(const uint8_t* tile, int r, int s, Vec8<float>& v)
 {
-    const float4* p = reinterpret_cast<const float4*>(tile + r * QTile<float>::row_bytes + s * 32);
-    v.a = p[0];
-    v.b = p[1];
+    const uint32_t a = smem_u32(tile) + r * QTile<float>::row_bytes + s * 32;
+    const uint4 x = lds_u4(a), y = lds_u4(a + 16);
+    v.a = make_float4(__uint_as_float(x.x), __uint_as_float(x.y), __uint_as_float(x.z), __uint_as_float(x.w));
+    v.b = make_float4(__uint_as_float(y.x), __uint_as_float(y.y), __uint_as_float(y.z), __uint_as_float(y.w));
 }
 
 template <typename T>

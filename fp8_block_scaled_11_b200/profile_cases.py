@@ -6,6 +6,7 @@ Cases (seeded inputs of the workloads, operands prepared before the loop so
 only the named kernel runs R times):
   gemm_fwd     Llama4 forward GEMM 16640 x 5120 x 8192, 1x128 x 128x128, bf16 out
   gemm_wgrad   Llama4 wgrad GEMM 5120 x 8192 x 16640, 1x128 x 1x128, bf16 out
+  gemm_dgrad   Llama4 dgrad GEMM 16640 x 8192 x 5120 (dy . W), 1x128 x 128x128, bf16 out
   gemm_tensor  16640 x 5120 x 8192 per-tensor scales, bf16 out
   gemm_longk   256 x 512 x 128128 (k_blocks 1001), 1x128 x 128x128, split-K, bf16 out
   quant_rows   1x128 quantization of a 32768 x 32768 bf16 matrix
@@ -39,6 +40,13 @@ def _gemm_case(name):
             mode = ops.SCALE_TENSOR
         out = torch.empty((M, 5120), dtype=torch.bfloat16, device="cuda")
         flops = 2.0 * M * 5120 * 8192
+    elif name == "gemm_dgrad":
+        _, W, dy = inputs.llama4(5120, 8192)
+        qa, sa = ops.fp8_quant_1x128(dy.cuda())
+        _, _, qb, sb = ops.fp8_quant_128x128(W.cuda(), want_q=False, want_qt=True)
+        mode = ops.SCALE_BLOCK_1x128_128x128
+        out = torch.empty((M, 8192), dtype=torch.bfloat16, device="cuda")
+        flops = 2.0 * M * 8192 * 5120
     elif name == "gemm_wgrad":
         x, _, dy = inputs.llama4(5120, 8192)
         qa, sa = ops.fp8_quant_1x128(dy.cuda(), transpose_out=True)

@@ -279,8 +279,9 @@ def test_llama4_fwd_bwd_workload(N, K):
 
 @pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("M", [129, 256, 257, 384, 512])
-def test_gemm_pair_tiles(M, mode):
-    """Row counts above 128 run on CTA pairs (256-row tiles): full pairs, a
-    pair whose second CTA is partly or wholly past the last row."""
+def test_gemm_several_tile_rows(M, mode):
+    """Row counts above 128: several 128-row tiles, the last one partly past
+    the last row."""
     run_random(M, 512, 384, mode, torch.float32, seed=M + 3 * mode)
     run_random(M, 264, 1024, mode, torch.bfloat16, seed=M + 5 * mode, guard=True)
+
