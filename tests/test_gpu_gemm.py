@@ -285,3 +285,24 @@ def test_gemm_several_tile_rows(M, mode):
     run_random(M, 512, 384, mode, torch.float32, seed=M + 3 * mode)
     run_random(M, 264, 1024, mode, torch.bfloat16, seed=M + 5 * mode, guard=True)
 
+
+
+@pytest.mark.parametrize("mode", [ops.SCALE_BLOCK_1x128_128x128, ops.SCALE_BLOCK_1x128_1x128])
+@pytest.mark.parametrize("M,N,K", [(1280, 2056, 256), (200, 520, 64 * 128)])
+def test_gemm_unaligned_output_pitch(M, N, K, mode):
+    """bf16 output into a view whose row pitch (N + 3 elements) is not a
+    multiple of 16 bytes, so every row is written element by element: by the
+    GEMM's epilogue (first shape: 90 tiles, no split) and by the split-K
+    reduction (second shape: 6 tiles, 64 K-blocks split 16 ways).  Parity on
+    all rows; nothing written outside the view."""
+    rng = np.random.default_rng(M + N)
+    A = inputs.random_e4m3_bytes(M, K, seed=M)
+    B = inputs.random_e4m3_bytes(N, K, seed=N)
+    sa, sb = make_scales(rng, mode, M, N, K)
+    buf = torch.full((M + 1, N + 3), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = buf[:M, :N]
+    ops.fp8_scaled_gemm(A.cuda(), B.cuda(), to_gpu_scales(sa, mode), to_gpu_scales(sb, mode), mode, out=out)
+    torch.cuda.synchronize()
+    no_device_error()
+    assert torch.isnan(buf[M:]).all() and torch.isnan(buf[:M, N:]).all(), "write outside the output view"
+    assert_bf16_close(out, oracle.gemm(A.numpy(), B.numpy(), sa, sb, mode), f"pitch N+3 M{M} N{N} K{K}")
