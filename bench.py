@@ -18,6 +18,7 @@ time is the max over ranks.  `--impl reference` times the CPU oracle instead
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -81,11 +82,14 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling: every 20 ms from start() to
+    stop(); only the samples whose timestamps fall inside the timed region
+    [t_begin, t_end] (host wall-clock seconds) are reported."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
@@ -95,7 +99,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -106,7 +110,34 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
+    @staticmethod
+    def parse(lines, t_begin, t_end):
+        """Median SM clock, max clock, median power and the throttle reasons
+        seen, over the samples taken inside [t_begin, t_end]."""
+        mhz, mx, pw, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, cmax, power = float(parts[2]), float(parts[3]), float(parts[4])
+            except ValueError:
+                continue
+            if not (t_begin <= ts <= t_end):
+                continue
+            mhz.append(clk)
+            mx.append(cmax)
+            pw.append(power)
+            for nm, v in zip(names, parts[6:10]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w": statistics.median(pw) if pw else None, "reasons": sorted(reasons),
+                "samples": len(mhz), "period_ms": ClockSampler.PERIOD_MS}
+
+    def stop(self, t_begin: float, t_end: float):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -115,22 +146,7 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.t.join(timeout=2)
-        mhz, mx, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                mhz.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+        return self.parse(self.lines, t_begin, t_end)
 
 
 # ------------------------------------------------------------------------ GPU arm
@@ -148,7 +164,6 @@ def run_gpu(args):
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
     if world > 1:
-        import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     ops.lib()
@@ -194,13 +209,15 @@ def run_gpu(args):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     events = []
+    wall0 = time.time()
     t0.record(stream)
     for _ in range(args.steps):
         one_step(events)
     t1.record(stream)
     torch.cuda.synchronize()
+    wall1 = time.time()
     barrier()
-    clocks = sampler.stop()
+    clocks = sampler.stop(wall0, wall1)
     ms_total = t0.elapsed_time(t1)
     quant_ms = sum(e[0].elapsed_time(e[1]) for _, e in events)
     gemm_ms = sum(e[1].elapsed_time(e[4]) for _, e in events)
