@@ -89,7 +89,7 @@ template <int MODE>
 struct EpiCfg {
     static constexpr int warps = MODE == kModeBlock1x128 ? 16 : 8;
     static constexpr bool reg_split = MODE == kModeBlock1x128 || MODE == kModeBlock128;
-    static constexpr bool single_buf = MODE == kModeBlock128;
+    static constexpr bool quad_loads = MODE == kModeBlock128;   // four TMEM loads per wait; else two in flight
     static constexpr int ctrl_warps = reg_split ? 4 : 2;
     static constexpr int threads = 32 * (ctrl_warps + warps);
     static constexpr int cols = kBN * 4 / warps;        // accumulator columns per thread
@@ -106,7 +106,7 @@ struct EpiCfg {
     static_assert(!reg_split || (ctrl_warps == 4 && warps % 4 == 0 &&
                                  128 * ctrl_regs + 32 * warps * epi_regs <= threads * launch_regs),
                   "register hand-over exceeds the launch allocation");
-    static_assert(!single_buf || chunks % 4 == 0, "four TMEM loads per wait");
+    static_assert(!quad_loads || chunks % 4 == 0, "four TMEM loads per wait");
 };
 
 struct GemmParams {
@@ -407,7 +407,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                             acc[c * 8 + j] = ffma2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), rowf2, acc[c * 8 + j]);
                     }
                 };
-                if constexpr (E::single_buf) {
+                if constexpr (E::quad_loads) {
                     // four 16-column loads per wait (64 registers in flight)
 #pragma unroll
                     for (int h = 0; h < kChunks / 4; ++h) {
