@@ -25,15 +25,18 @@ __device__ int g_device_error;
 
 constexpr int kMaxDevices = 64;
 
+// Per-device state, filled on first use.  Calls may come from several host
+// threads: the flags are atomics (release on set, acquire on test) and every
+// first-time set-up runs under g_mutex.
 struct DeviceInfo {
-    bool ready = false;
+    std::atomic<bool> ready{false};
     bool sm100 = false;
     int num_sms = 0;
     int* err_ptr = nullptr;
-    bool gemm_attr_set[4] = {false, false, false, false};
-    int quant_blocks[10] = {0};  // resident CTAs per SM, per quant kernel kind
-    bool tile_attr_set[6] = {false, false, false, false, false, false};
-    int tile_blocks[6] = {0};
+    std::atomic<bool> gemm_attr_set[4]{};
+    std::atomic<int> quant_blocks[10]{};     // resident CTAs per SM, per quant kernel kind
+    std::atomic<bool> tile_attr_set[6]{};
+    std::atomic<int> tile_blocks[6]{};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -49,9 +52,9 @@ fp8bs_status get_device(DeviceInfo** out)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8BS_ERR_CUDA;
     DeviceInfo& d = g_dev[dev];
-    if (!d.ready) {
+    if (!d.ready.load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(g_mutex);
-        if (!d.ready) {
+        if (!d.ready.load(std::memory_order_relaxed)) {
             int major = 0;
             if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return FP8BS_ERR_CUDA;
             d.sm100 = (major == 10);
@@ -69,7 +72,7 @@ fp8bs_status get_device(DeviceInfo** out)
                     return FP8BS_ERR_CUDA;
                 g_encode = reinterpret_cast<EncodeTiledFn>(fn);
             }
-            d.ready = true;
+            d.ready.store(true, std::memory_order_release);
         }
     }
     if (!d.sm100) return FP8BS_ERR_NO_SM100;
@@ -91,12 +94,13 @@ fp8bs_status launch_status()
 template <typename Kernel>
 int persistent_grid(DeviceInfo* d, int kind, Kernel k, int64_t work_ctas)
 {
-    if (d->quant_blocks[kind] == 0) {
-        int nb = 0;
+    int nb = d->quant_blocks[kind].load(std::memory_order_acquire);
+    if (nb == 0) {
+        // racing first calls compute the same value
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k, 256, 0) != cudaSuccess || nb < 1) nb = 1;
-        d->quant_blocks[kind] = nb;
+        d->quant_blocks[kind].store(nb, std::memory_order_release);
     }
-    const int64_t cap = (int64_t)d->quant_blocks[kind] * d->num_sms;
+    const int64_t cap = (int64_t)nb * d->num_sms;
     return (int)std::max<int64_t>(1, std::min<int64_t>(cap, work_ctas));
 }
 
@@ -106,15 +110,19 @@ template <typename Kernel, typename... Args>
 fp8bs_status launch_tile_kernel(DeviceInfo* d, int kind, Kernel k, uint32_t smem, int64_t tiles, cudaStream_t stream,
                                 Args... args)
 {
-    if (!d->tile_attr_set[kind]) {
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return FP8BS_ERR_CUDA;
-        int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k, 256, smem) != cudaSuccess || nb < 1) nb = 1;
-        d->tile_blocks[kind] = nb;
-        d->tile_attr_set[kind] = true;
+    if (!d->tile_attr_set[kind].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!d->tile_attr_set[kind].load(std::memory_order_relaxed)) {
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+                return FP8BS_ERR_CUDA;
+            int nb = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k, 256, smem) != cudaSuccess || nb < 1) nb = 1;
+            d->tile_blocks[kind].store(nb, std::memory_order_relaxed);
+            d->tile_attr_set[kind].store(true, std::memory_order_release);
+        }
     }
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)d->tile_blocks[kind] * d->num_sms));
+    const int64_t per_sm = d->tile_blocks[kind].load(std::memory_order_relaxed);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, per_sm * d->num_sms));
     k<<<grid, 256, smem, stream>>>(args...);
     return launch_status();
 }
@@ -172,18 +180,22 @@ fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap
                          const CUtensorMap& tSB, const GemmParams& p, cudaStream_t stream)
 {
     auto k = gemm_fp8_kernel<MODE>;
-    if (!d->gemm_attr_set[MODE]) {
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::alloc) != cudaSuccess)
-            return FP8BS_ERR_CUDA;
-        if (EpiCfg<MODE>::reg_split) {
-            // the warpgroups' register hand-over is sized for this exact
-            // allocation at launch; with fewer registers the promotion warps'
-            // increase could never be granted, so refuse to launch instead
-            cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return FP8BS_ERR_CUDA;
-            if (fa.numRegs != EpiCfg<MODE>::launch_regs) return FP8BS_ERR_UNSUPPORTED;
+    if (!d->gemm_attr_set[MODE].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!d->gemm_attr_set[MODE].load(std::memory_order_relaxed)) {
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::alloc) !=
+                cudaSuccess)
+                return FP8BS_ERR_CUDA;
+            if (EpiCfg<MODE>::reg_split) {
+                // the warpgroups' register hand-over is sized for this exact
+                // allocation at launch; with fewer registers the promotion warps'
+                // increase could never be granted, so refuse to launch instead
+                cudaFuncAttributes fa;
+                if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return FP8BS_ERR_CUDA;
+                if (fa.numRegs != EpiCfg<MODE>::launch_regs) return FP8BS_ERR_UNSUPPORTED;
+            }
+            d->gemm_attr_set[MODE].store(true, std::memory_order_release);
         }
-        d->gemm_attr_set[MODE] = true;
     }
     const int grid = (int)std::min<int64_t>(p.num_units, d->num_sms);
     k<<<grid, EpiCfg<MODE>::threads, SmemLayout::alloc, stream>>>(tA, tB, tSA, tSB, p);
@@ -563,7 +575,7 @@ namespace {
 constexpr int kNoAllocPartials = 4096;                  // floats of scratch (16 KB)
 constexpr int64_t kNoAllocElemsPerPartial = 65536;      // elements reduced per amax CTA
 constexpr int64_t kNoAllocMaxElems = (int64_t)kNoAllocPartials * kNoAllocElemsPerPartial;
-float* g_noalloc_scratch[kMaxDevices] = {nullptr};      // device address of the array, per device
+std::atomic<float*> g_noalloc_scratch[kMaxDevices]{};   // device address of the array, per device
 std::mutex g_noalloc_mutex;
 }  // namespace
 
@@ -584,16 +596,18 @@ extern "C" fp8bs_status fp8_quant_tensor_noalloc(const void* x, fp8bs_dtype xt, 
     if (st != FP8BS_OK) return st;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP8BS_ERR_CUDA;
-    if (g_noalloc_scratch[dev] == nullptr) {
+    float* partial = g_noalloc_scratch[dev].load(std::memory_order_acquire);
+    if (partial == nullptr) {
         // one-time set-up per device, with that device current
         std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-        if (g_noalloc_scratch[dev] == nullptr) {
+        partial = g_noalloc_scratch[dev].load(std::memory_order_relaxed);
+        if (partial == nullptr) {
             void* p = nullptr;
             if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || p == nullptr) return FP8BS_ERR_CUDA;
-            g_noalloc_scratch[dev] = static_cast<float*>(p);
+            partial = static_cast<float*>(p);
+            g_noalloc_scratch[dev].store(partial, std::memory_order_release);
         }
     }
-    float* partial = g_noalloc_scratch[dev];
     // every partial slot the second kernel reads is written by the first one in
     // this same call, so nothing left by an earlier call needs clearing
     const int parts = (int)std::max<int64_t>(1, cdiv(n, kNoAllocElemsPerPartial));
