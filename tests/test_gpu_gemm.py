@@ -306,3 +306,48 @@ def test_gemm_unaligned_output_pitch(M, N, K, mode):
     no_device_error()
     assert torch.isnan(buf[M:]).all() and torch.isnan(buf[:M, N:]).all(), "write outside the output view"
     assert_bf16_close(out, oracle.gemm(A.numpy(), B.numpy(), sa, sb, mode), f"pitch N+3 M{M} N{N} K{K}")
+
+
+def test_llama4_forward_fp32_output_sampled():
+    """The forward GEMM at full size (16640 x 5120 x 8192, 1x128 x 128x128) with
+    fp32 output, in the benchmark's launch configuration: sampled rows from
+    the first, middle and last tile rows against the oracle (relative
+    Frobenius error <= 1e-5)."""
+    M = inputs.LLAMA4_M
+    x, W, _ = inputs.llama4(5120, 8192)
+    xd, Wd = x.cuda(), W.cuda()
+    qx, sx = ops.fp8_quant_1x128(xd)
+    qw, sw, _, _ = ops.fp8_quant_128x128(Wd)
+    D = ops.fp8_scaled_gemm(qx, qw, sx, sw, ops.SCALE_BLOCK_1x128_128x128, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    no_device_error()
+    rows = [0, 77, 128, 8191, 8320, M - 129, M - 1]
+    qxo, sxo = oracle.quant_1x128(bits(x), rows=rows)
+    qwo, swo = oracle.quant_128x128(bits(W))
+    ref = oracle.gemm(qxo, qwo, sxo, swo, oracle.SCALE_BLOCK_1x128_128x128)
+    assert_f32_close(D[torch.as_tensor(rows, device="cuda")], ref, "fwd fp32 out")
+
+
+@pytest.mark.parametrize("recipe", ["1x128_128x128", "1x128_1x128"])
+def test_long_k_fp32_output(recipe):
+    """The long-K case at k_blocks 1001 with fp32 output (split-K reduction
+    writing fp32): sampled rows of both 128-row tiles against the oracle."""
+    K = 128128
+    goT, x = inputs.long_k(K)
+    goTd, xd = goT.cuda(), x.cuda()
+    qa, sa = ops.fp8_quant_1x128(goTd)
+    if recipe == "1x128_128x128":
+        _, _, qb, sb = ops.fp8_quant_128x128(xd, want_q=False, want_qt=True)
+        mode = ops.SCALE_BLOCK_1x128_128x128
+        qbo, sbo = oracle.quant_128x128(bits(x), transpose=True)
+    else:
+        qb, sb = ops.fp8_quant_1x128(xd, transpose_out=True)
+        mode = ops.SCALE_BLOCK_1x128_1x128
+        qbo, sbo = oracle.quant_1x128(bits(x), transpose=True)
+    D = ops.fp8_scaled_gemm(qa, qb, sa, sb, mode, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    no_device_error()
+    rows = [0, 5, 64, 127, 128, 191, 255]
+    qao, sao = oracle.quant_1x128(bits(goT), rows=rows)
+    assert_f32_close(D[torch.as_tensor(rows, device="cuda")], oracle.gemm(qao, qbo, sao, sbo, mode),
+                     f"long K fp32 out {recipe}")
