@@ -35,8 +35,8 @@ struct DeviceInfo {
     int* err_ptr = nullptr;
     std::atomic<bool> gemm_attr_set[4]{};
     std::atomic<int> quant_blocks[10]{};     // resident CTAs per SM, per quant kernel kind
-    std::atomic<bool> tile_attr_set[6]{};
-    std::atomic<int> tile_blocks[6]{};
+    std::atomic<bool> tile_attr_set[8]{};
+    std::atomic<int> tile_blocks[8]{};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -158,8 +158,9 @@ SplitPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms)
     const int64_t Kb = cdiv(K, kBK);
     int splits = 1;
     if (tiles * 2 <= num_sms) {
-        // fill the SMs, but keep >= 4 K-blocks per split so the pipeline runs
-        splits = (int)std::min<int64_t>(num_sms / tiles, std::max<int64_t>(1, Kb / 4));
+        // fill the SMs, but keep >= 8 K-blocks per split: with fewer, the
+        // pipeline fill and the reduction's extra launch outweigh the split
+        splits = (int)std::min<int64_t>(num_sms / tiles, std::max<int64_t>(1, Kb / 8));
         splits = std::max(1, std::min(splits, 64));
     }
     s.splits = splits;
@@ -256,7 +257,25 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
     fp8bs_status st = get_device(&d);
     if (st != FP8BS_OK) return st;
 
-    if (!transpose_out) {
+    if (!transpose_out && rows % 16 == 0) {
+        // whole 16-row blocks: the TMA tile pipeline (higher HBM throughput)
+        const int64_t ctas = cdiv(rows, 128) * cdiv(cols, 128);
+        CUtensorMap map;
+        if (xt == FP8BS_BF16) {
+            if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, ldx * 2, 128, 128,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
+                return st;
+            st = launch_tile_kernel(d, 6, quant_1x128_rowtile_kernel<__nv_bfloat16>, QTile<__nv_bfloat16>::smem, ctas,
+                                    stream, map, rows, cols, q, ldq, scale_inv, ld_scale, d->err_ptr);
+        } else {
+            if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, x, cols, rows, ldx * 4, 128, 128,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
+                return st;
+            st = launch_tile_kernel(d, 7, quant_1x128_rowtile_kernel<float>, QTile<float>::smem, ctas, stream, map,
+                                    rows, cols, q, ldq, scale_inv, ld_scale, d->err_ptr);
+        }
+        if (st != FP8BS_OK) return st;
+    } else if (!transpose_out) {
         const int64_t items = cdiv(rows, 32) * cdiv(cols, 128);
         const int64_t ctas = cdiv(items, 8);
         if (xt == FP8BS_BF16) {

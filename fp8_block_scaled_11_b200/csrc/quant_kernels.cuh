@@ -365,6 +365,66 @@ __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(
     });
 }
 
+// 1x128 groups along the contiguous dimension, through the tile pipeline: a
+// 128 x 128 tile holds 128 whole row groups; row maxima over the thread's 8
+// columns, the warp's 8 strips (shuffles) and the tile's two 64-column halves
+// (shared memory).  Byte-identical to quant_1x128_rows_kernel; used when the
+// row count is a multiple of 16.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_1x128_rowtile_kernel(
+    const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
+    uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sinv, int64_t ld_s, int* err)
+{
+    __shared__ float s_rpart[2][128];                 // row maxima per 64-column half
+    __shared__ float s_rscale[128];
+    int strip, group, wr, wc;
+    qblock_coords(strip, group, wr, wc);
+    const int lane = threadIdx.x & 31;
+    const int64_t tiles_c = (cols + 127) >> 7;
+    const int64_t ntiles = ((rows + 127) >> 7) * tiles_c;
+    tile_pipeline<T>(&map, ntiles, tiles_c, err, [&](const uint8_t* tile, int64_t t, auto&& release) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        Block8x8<T> blk;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lds_vec8<T>(tile, 8 * group + i, strip, blk.row[i]);
+        float rm[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float f[8];
+            blk.row[i].get(f);
+            rm[i] = absmax8(f);
+            rm[i] = fmaxf(rm[i], __shfl_xor_sync(0xffffffffu, rm[i], 1));
+            rm[i] = fmaxf(rm[i], __shfl_xor_sync(0xffffffffu, rm[i], 2));
+            rm[i] = fmaxf(rm[i], __shfl_xor_sync(0xffffffffu, rm[i], 4));
+        }
+        if ((lane & 7) == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s_rpart[wc][8 * group + i] = rm[i];
+        }
+        __syncthreads();
+        release();
+        if (threadIdx.x < 128) {
+            const int r = threadIdx.x;
+            const float sr = scale_from_amax(fmaxf(s_rpart[0][r], s_rpart[1][r]));
+            s_rscale[r] = sr;
+            const int64_t rg = (tr << 7) + r;
+            if (rg < rows) sinv[rg + tc * ld_s] = __frcp_rn(sr);
+        }
+        __syncthreads();
+        const int64_t r0 = (tr << 7) + 8 * group;
+        const int64_t c0 = (tc << 7) + 8 * strip;
+        if (c0 < cols && r0 < rows) {          // rows, cols % 16 == 0: 8-blocks are all-in or all-out
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float f[8];
+                blk.row[i].get(f);
+                *reinterpret_cast<uint2*>(q + (r0 + i) * ldq + c0) = quant8(f, s_rscale[8 * group + i]);
+            }
+        }
+        __syncthreads();                       // the shared arrays are rewritten by the next tile
+    });
+}
+
 // Both 1x128 directions from one read of the input.  A 128 x 128 tile holds
 // 128 whole row groups (1x128 along the columns) and 128 whole column groups
 // (1x128 along the rows), so one pass over the tile gives both sets of

@@ -13,7 +13,16 @@ only the named kernel runs R times):
   quant_cols   1x128 along rows (transposed output) of a 16640 x 8192 bf16 matrix
   quant_dual   both 1x128 directions from one read of a 16640 x 8192 bf16 matrix
   quant_tile   128x128 quantization (with transposed copy) of a 32768 x 32768 bf16 matrix
+  gemm_tiny            256 x 512 x 1024, 1x128 x 128x128, bf16 out (the tiny blockwise case)
+  gemm_pertensor_small 256 x 4096 x 1024 per-tensor scales, bf16 out
+  gemm_rowwise_small   256 x 4096 x 1024 rowwise scales, bf16 out
+  quant_rows_<n>, quant_tile_<n>   the quantization sweep at n x n bf16 (n = 1024 ... 32768)
 With --time, each launch is timed with CUDA events and the mean is printed.
+
+  python -m fp8_block_scaled_11_b200.profile_cases configs [--reps R]
+
+times every case above (the median of three rounds of R timed launches each)
+and prints one table.
 """
 from __future__ import annotations
 
@@ -27,7 +36,25 @@ from . import inputs, ops
 
 def _gemm_case(name):
     M = inputs.LLAMA4_M
-    if name in ("gemm_fwd", "gemm_tensor"):
+    if name == "gemm_tiny":
+        A, Bt = inputs.tiny_blockwise()
+        qa, sa = ops.fp8_quant_1x128(A.cuda())
+        qb, sb, _, _ = ops.fp8_quant_128x128(Bt.cuda())
+        mode = ops.SCALE_BLOCK_1x128_128x128
+        out = torch.empty((256, 512), dtype=torch.bfloat16, device="cuda")
+        flops = 2.0 * 256 * 512 * 1024
+    elif name in ("gemm_pertensor_small", "gemm_rowwise_small"):
+        x, W = inputs.per_tensor()
+        xd, Wd = x.cuda(), W.cuda()
+        if name == "gemm_pertensor_small":
+            (qa, sa), (qb, sb) = ops.fp8_quant_tensor(xd), ops.fp8_quant_tensor(Wd)
+            mode = ops.SCALE_TENSOR
+        else:
+            (qa, sa), (qb, sb) = ops.fp8_quant_rowwise(xd), ops.fp8_quant_rowwise(Wd)
+            mode = ops.SCALE_ROWWISE
+        out = torch.empty((256, 4096), dtype=torch.bfloat16, device="cuda")
+        flops = 2.0 * 256 * 4096 * 1024
+    elif name in ("gemm_fwd", "gemm_tensor"):
         x, W, _ = inputs.llama4(5120, 8192)
         x, W = x.cuda(), W.cuda()
         if name == "gemm_fwd":
@@ -68,6 +95,21 @@ def _gemm_case(name):
 
 
 def _quant_case(name):
+    parts = name.split("_")
+    if len(parts) == 3 and parts[2].isdigit():
+        # the quantization sweep: quant_rows_<n> / quant_tile_<n>
+        n = int(parts[2])
+        x = inputs.quant_sweep(n).cuda()
+        if parts[1] == "rows":
+            q, s = ops.fp8_quant_1x128(x)
+            nbytes = x.numel() * 3 + 4 * s.numel()
+            fn = lambda: ops.fp8_quant_1x128(x, q=q, scale_inv=s)
+        else:
+            out = ops.fp8_quant_128x128(x)
+            nbytes = x.numel() * 3 + 4 * out[1].numel()
+            fn = lambda: ops.fp8_quant_128x128(x, out=out)
+        torch.cuda.synchronize()
+        return fn, nbytes, "GB/s"
     if name == "quant_cols":
         x = inputs.llama4(5120, 8192)[0].cuda()
         q, s = ops.fp8_quant_1x128(x, transpose_out=True)
@@ -92,12 +134,49 @@ def _quant_case(name):
     return fn, nbytes, "GB/s"
 
 
+CONFIG_CASES = (["gemm_tiny", "gemm_pertensor_small", "gemm_rowwise_small", "gemm_fwd", "gemm_dgrad",
+                 "gemm_wgrad", "gemm_tensor", "gemm_longk", "quant_dual"]
+                + [f"quant_rows_{n}" for n in inputs.QUANT_SWEEP_SIZES]
+                + [f"quant_tile_{n}" for n in inputs.QUANT_SWEEP_SIZES])
+
+
+def _time(case, reps):
+    fn, work, unit = _gemm_case(case) if case.startswith("gemm") else _quant_case(case)
+    fn()
+    torch.cuda.synchronize()
+    rounds = []
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        rounds.append(a.elapsed_time(b) / reps)
+    st = ops.fp8bs_check_device_error()
+    if st != 0:
+        raise RuntimeError(f"{case}: {ops.fp8bs_status_string(st)}")
+    ms = sorted(rounds)[1]
+    return ms, work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9), unit
+
+
+def configs(reps):
+    print(f"{'case':22s} {'us/launch':>10s} {'rate':>10s}")
+    for case in CONFIG_CASES:
+        ms, rate, unit = _time(case, reps)
+        print(f"{case:22s} {ms * 1e3:10.1f} {rate:10.1f} {unit}")
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("case")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--time", action="store_true")
     a = ap.parse_args(argv)
+    if a.case == "configs":
+        return configs(a.reps)
     if a.case.startswith("gemm"):
         fn, work, unit = _gemm_case(a.case)
     else:

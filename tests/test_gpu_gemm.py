@@ -293,7 +293,7 @@ def test_gemm_unaligned_output_pitch(M, N, K, mode):
     """bf16 output into a view whose row pitch (N + 3 elements) is not a
     multiple of 16 bytes, so every row is written element by element: by the
     GEMM's epilogue (first shape: 90 tiles, no split) and by the split-K
-    reduction (second shape: 6 tiles, 64 K-blocks split 16 ways).  Parity on
+    reduction (second shape: 6 tiles, 64 K-blocks split 8 ways).  Parity on
     all rows; nothing written outside the view."""
     rng = np.random.default_rng(M + N)
     A = inputs.random_e4m3_bytes(M, K, seed=M)
