@@ -105,6 +105,12 @@ class ClockSampler:
             self.t.start()
         except OSError:
             self.proc = None
+            return
+        # the timed region starts only once samples are flowing (nvidia-smi can
+        # take a while to print its first one)
+        t_end = time.time() + 5.0
+        while len(self.lines) < 2 and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -203,7 +209,6 @@ def run_gpu(args):
     # ---- timed region: K steps, CUDA events on the launching stream
     sampler = ClockSampler(local)
     sampler.start()
-    time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
