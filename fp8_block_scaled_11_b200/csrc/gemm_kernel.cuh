@@ -11,8 +11,10 @@
 // One persistent CTA per SM computes 128 x 256 output tiles:
 //   warp 0      TMA producer: per K-block one 128x128 tile of A and one
 //               256x128 tile of B^T (bytes, 128-byte swizzle) into a 4-stage
-//               shared-memory ring, and the K-block's scale vectors into a
-//               separate ring (they are read later, by the promotion warps).
+//               shared-memory ring; for the rowwise and 1x128 x 1x128 recipes
+//               also the K-block's scale vectors into a separate ring (the
+//               1x128 x 128x128 promotion warps read their two scalars per
+//               K-block from L2 themselves).
 //   warp 1      TMEM allocation; lane 0 issues four tcgen05.mma (128x256x32,
 //               e4m3 x e4m3 -> fp32) per K-block into one of two 256-column
 //               TMEM accumulators and commits the accumulator and the smem
