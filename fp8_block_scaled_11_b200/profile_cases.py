@@ -8,6 +8,7 @@ only the named kernel runs R times):
   gemm_wgrad   Llama4 wgrad GEMM 5120 x 8192 x 16640, 1x128 x 1x128, bf16 out
   gemm_dgrad   Llama4 dgrad GEMM 16640 x 8192 x 5120 (dy . W), 1x128 x 128x128, bf16 out
   gemm_tensor  16640 x 5120 x 8192 per-tensor scales, bf16 out
+  gemm_rowwise 16640 x 5120 x 8192 rowwise scales, bf16 out
   gemm_longk   256 x 512 x 128128 (k_blocks 1001), 1x128 x 128x128, split-K, bf16 out
   quant_rows   1x128 quantization of a 32768 x 32768 bf16 matrix
   quant_cols   1x128 along rows (transposed output) of a 16640 x 8192 bf16 matrix
@@ -54,13 +55,16 @@ def _gemm_case(name):
             mode = ops.SCALE_ROWWISE
         out = torch.empty((256, 4096), dtype=torch.bfloat16, device="cuda")
         flops = 2.0 * 256 * 4096 * 1024
-    elif name in ("gemm_fwd", "gemm_tensor"):
+    elif name in ("gemm_fwd", "gemm_tensor", "gemm_rowwise"):
         x, W, _ = inputs.llama4(5120, 8192)
         x, W = x.cuda(), W.cuda()
         if name == "gemm_fwd":
             qa, sa = ops.fp8_quant_1x128(x)
             qb, sb, _, _ = ops.fp8_quant_128x128(W)
             mode = ops.SCALE_BLOCK_1x128_128x128
+        elif name == "gemm_rowwise":
+            (qa, sa), (qb, sb) = ops.fp8_quant_rowwise(x), ops.fp8_quant_rowwise(W)
+            mode = ops.SCALE_ROWWISE
         else:
             qa, sa = ops.fp8_quant_tensor(x)
             qb, sb = ops.fp8_quant_tensor(W)
@@ -135,7 +139,7 @@ def _quant_case(name):
 
 
 CONFIG_CASES = (["gemm_tiny", "gemm_pertensor_small", "gemm_rowwise_small", "gemm_fwd", "gemm_dgrad",
-                 "gemm_wgrad", "gemm_tensor", "gemm_longk", "quant_dual"]
+                 "gemm_wgrad", "gemm_tensor", "gemm_rowwise", "gemm_longk", "quant_dual"]
                 + [f"quant_rows_{n}" for n in inputs.QUANT_SWEEP_SIZES]
                 + [f"quant_tile_{n}" for n in inputs.QUANT_SWEEP_SIZES])
 
