@@ -33,7 +33,7 @@ struct DeviceInfo {
     bool sm100 = false;
     int num_sms = 0;
     int* err_ptr = nullptr;
-    std::atomic<bool> gemm_attr_set[4]{};
+    std::atomic<bool> gemm_attr_set[8]{};    // per recipe, without / with the fused output quantization
     std::atomic<int> quant_blocks[10]{};     // resident CTAs per SM, per quant kernel kind
     std::atomic<bool> tile_attr_set[8]{};
     std::atomic<int> tile_blocks[8]{};
@@ -176,14 +176,16 @@ int num_sms_current()
     return d->num_sms;
 }
 
-template <int MODE>
+template <int MODE, bool QOUT = false>
 fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA,
-                         const CUtensorMap& tSB, const GemmParams& p, cudaStream_t stream)
+                         const CUtensorMap& tSB, const std::conditional_t<QOUT, GemmParamsQ, GemmParams>& p,
+                         cudaStream_t stream)
 {
-    auto k = gemm_fp8_kernel<MODE>;
-    if (!d->gemm_attr_set[MODE].load(std::memory_order_acquire)) {
+    auto k = gemm_fp8_kernel<MODE, QOUT>;
+    constexpr int slot = MODE + (QOUT ? 4 : 0);
+    if (!d->gemm_attr_set[slot].load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(g_mutex);
-        if (!d->gemm_attr_set[MODE].load(std::memory_order_relaxed)) {
+        if (!d->gemm_attr_set[slot].load(std::memory_order_relaxed)) {
             if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SmemLayout::alloc) !=
                 cudaSuccess)
                 return FP8BS_ERR_CUDA;
@@ -195,7 +197,7 @@ fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap
                 if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return FP8BS_ERR_CUDA;
                 if (fa.numRegs != EpiCfg<MODE>::launch_regs) return FP8BS_ERR_UNSUPPORTED;
             }
-            d->gemm_attr_set[MODE].store(true, std::memory_order_release);
+            d->gemm_attr_set[slot].store(true, std::memory_order_release);
         }
     }
     const int grid = (int)std::min<int64_t>(p.num_units, d->num_sms);
@@ -452,17 +454,37 @@ size_t fp8_scaled_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8bs_sca
     return plan_gemm(M, N, K, num_sms_current()).ws_bytes;
 }
 
-fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* Bt,
-                             int64_t ldb, const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
-                             fp8bs_scale_mode mode, fp8bs_scale_layout layout, void* D, int64_t ldd,
-                             fp8bs_dtype out_dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+// Output quantization requested by fp8_scaled_gemm_quant (q == nullptr: none).
+struct QuantOut {
+    uint8_t* q = nullptr;
+    int64_t ldq = 0;
+    float* s = nullptr;
+    int64_t lds = 0;
+};
+
+fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* Bt,
+                         int64_t ldb, const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
+                         fp8bs_scale_mode mode, fp8bs_scale_layout layout, void* D, int64_t ldd,
+                         fp8bs_dtype out_dtype, void* workspace, size_t workspace_bytes, const QuantOut& qo,
+                         cudaStream_t stream)
 {
+    const bool quant_out = qo.q != nullptr;
     if (mode < FP8BS_SCALE_TENSOR || mode > FP8BS_SCALE_BLOCK_1x128_1x128) return FP8BS_ERR_UNSUPPORTED;
     if (layout != FP8BS_SCALE_COL_MAJOR || !valid_dtype(out_dtype)) return FP8BS_ERR_UNSUPPORTED;
-    if (A == nullptr || Bt == nullptr || scale_a == nullptr || scale_b == nullptr || D == nullptr) return FP8BS_ERR_INVALID_ARG;
+    if (quant_out && (mode == FP8BS_SCALE_BLOCK_1x128_1x128 || out_dtype != FP8BS_BF16)) return FP8BS_ERR_UNSUPPORTED;
+    if (A == nullptr || Bt == nullptr || scale_a == nullptr || scale_b == nullptr) return FP8BS_ERR_INVALID_ARG;
+    if (D == nullptr && !quant_out) return FP8BS_ERR_INVALID_ARG;
     if (M < 1 || N < 1 || K < 16) return FP8BS_ERR_INVALID_ARG;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8BS_ERR_INVALID_ARG;
-    if (lda < K || ldb < K || ldd < N) return FP8BS_ERR_INVALID_ARG;
+    if (lda < K || ldb < K || (D != nullptr && ldd < N)) return FP8BS_ERR_INVALID_ARG;
+    if (quant_out) {
+        if (qo.s == nullptr || qo.ldq < N || qo.lds < M) return FP8BS_ERR_INVALID_ARG;
+        if (!aligned16(qo.q) || !aligned16(qo.s) || qo.ldq % 16 || qo.lds % 4) return FP8BS_ERR_ALIGNMENT;
+    }
     const int64_t Kb = cdiv(K, kBK), Nb = cdiv(N, 128);
     const bool block = (mode == FP8BS_SCALE_BLOCK_1x128_128x128 || mode == FP8BS_SCALE_BLOCK_1x128_1x128);
     if (block) {
@@ -474,12 +496,13 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
     if (K % 16 || lda % 16 || ldb % 16) return FP8BS_ERR_ALIGNMENT;
     if (!aligned16(A) || !aligned16(Bt) || !aligned16(scale_a) || !aligned16(scale_b)) return FP8BS_ERR_ALIGNMENT;
     if (reinterpret_cast<uintptr_t>(D) % dtype_size(out_dtype)) return FP8BS_ERR_ALIGNMENT;
-    const int vec_out = aligned16(D) && (ldd * (int64_t)dtype_size(out_dtype)) % 16 == 0;
+    const int vec_out = D != nullptr && aligned16(D) && (ldd * (int64_t)dtype_size(out_dtype)) % 16 == 0;
     DeviceInfo* d = nullptr;
     fp8bs_status st = get_device(&d);
     if (st != FP8BS_OK) return st;
 
     SplitPlan plan = plan_gemm(M, N, K, d->num_sms);
+    if (quant_out) plan.splits = 1;              // the epilogue quantizes whole tiles
     if (plan.splits > 1) {
         if (workspace == nullptr && workspace_bytes == 0) {
             plan.splits = 1;                     // split-K disabled by the caller
@@ -513,7 +536,7 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
         break;
     }
 
-    GemmParams p;
+    GemmParamsQ p;
     p.M = (int32_t)M;
     p.N = (int32_t)N;
     p.K = (int32_t)K;
@@ -534,12 +557,24 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
     p.ld_sa = ld_sa;
     p.ld_sb = ld_sb;
     p.err = d->err_ptr;
+    p.qout = qo.q;
+    p.ldq_out = qo.ldq;
+    p.sout = qo.s;
+    p.lds_out = qo.lds;
 
+    if (quant_out) {
+        switch (mode) {
+        case FP8BS_SCALE_TENSOR: return launch_gemm<kModeTensor, true>(d, tA, tB, tSA, tSB, p, stream);
+        case FP8BS_SCALE_ROWWISE: return launch_gemm<kModeRowwise, true>(d, tA, tB, tSA, tSB, p, stream);
+        default: return launch_gemm<kModeBlock128, true>(d, tA, tB, tSA, tSB, p, stream);
+        }
+    }
+    const GemmParams& pb = p;                    // the plain instantiations take the base block
     switch (mode) {
-    case FP8BS_SCALE_TENSOR: st = launch_gemm<kModeTensor>(d, tA, tB, tSA, tSB, p, stream); break;
-    case FP8BS_SCALE_ROWWISE: st = launch_gemm<kModeRowwise>(d, tA, tB, tSA, tSB, p, stream); break;
-    case FP8BS_SCALE_BLOCK_1x128_128x128: st = launch_gemm<kModeBlock128>(d, tA, tB, tSA, tSB, p, stream); break;
-    case FP8BS_SCALE_BLOCK_1x128_1x128: st = launch_gemm<kModeBlock1x128>(d, tA, tB, tSA, tSB, p, stream); break;
+    case FP8BS_SCALE_TENSOR: st = launch_gemm<kModeTensor>(d, tA, tB, tSA, tSB, pb, stream); break;
+    case FP8BS_SCALE_ROWWISE: st = launch_gemm<kModeRowwise>(d, tA, tB, tSA, tSB, pb, stream); break;
+    case FP8BS_SCALE_BLOCK_1x128_128x128: st = launch_gemm<kModeBlock128>(d, tA, tB, tSA, tSB, pb, stream); break;
+    case FP8BS_SCALE_BLOCK_1x128_1x128: st = launch_gemm<kModeBlock1x128>(d, tA, tB, tSA, tSB, pb, stream); break;
     }
     if (st != FP8BS_OK) return st;
     if (plan.splits > 1) {
@@ -551,6 +586,36 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
         st = launch_status();
     }
     return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* Bt,
+                             int64_t ldb, const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
+                             fp8bs_scale_mode mode, fp8bs_scale_layout layout, void* D, int64_t ldd,
+                             fp8bs_dtype out_dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (D == nullptr) return FP8BS_ERR_INVALID_ARG;
+    return scaled_gemm(M, N, K, A, lda, Bt, ldb, scale_a, ld_sa, scale_b, ld_sb, mode, layout, D, ldd, out_dtype,
+                       workspace, workspace_bytes, QuantOut{}, stream);
+}
+
+fp8bs_status fp8_scaled_gemm_quant(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* Bt,
+                                   int64_t ldb, const float* scale_a, int64_t ld_sa, const float* scale_b,
+                                   int64_t ld_sb, fp8bs_scale_mode mode, fp8bs_scale_layout layout, void* D,
+                                   int64_t ldd, uint8_t* q_out, int64_t ldq_out, float* scale_out,
+                                   int64_t ld_scale_out, cudaStream_t stream)
+{
+    if (q_out == nullptr) return FP8BS_ERR_INVALID_ARG;
+    QuantOut qo;
+    qo.q = q_out;
+    qo.ldq = ldq_out;
+    qo.s = scale_out;
+    qo.lds = ld_scale_out;
+    return scaled_gemm(M, N, K, A, lda, Bt, ldb, scale_a, ld_sa, scale_b, ld_sb, mode, layout, D, ldd, FP8BS_BF16,
+                       nullptr, 0, qo, stream);
 }
 
 }  // extern "C"

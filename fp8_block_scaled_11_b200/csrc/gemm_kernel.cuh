@@ -42,9 +42,11 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include "ptx.cuh"
+#include "quant_kernels.cuh"
 
 namespace fp8bs {
 
@@ -130,6 +132,16 @@ struct GemmParams {
     int* err;                   // library error flag
 };
 
+// The fused-quantization instantiation's parameters: the bf16 output's 1x128
+// groups along N as e4m3 bytes and reciprocal scales.  (A separate type, so
+// that the other instantiations keep their parameter block as it is.)
+struct GemmParamsQ : GemmParams {
+    uint8_t* qout;
+    int64_t ldq_out;
+    float* sout;
+    int64_t lds_out;
+};
+
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int64_t u, int& tm, int& tn, int& kb0, int& kb1,
                                             int& split)
 {
@@ -147,13 +159,17 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int64_t u, int&
     kb1 = (int)(((int64_t)p.Kb * (split + 1)) / p.splits);
 }
 
-template <int MODE>
+// QOUT: the epilogue also quantizes the bf16 output, 1x128 along N (each
+// promotion thread holds one row's 128 consecutive columns: one whole group),
+// byte-identical to quantizing the stored bf16 output afterwards.
+template <int MODE, bool QOUT = false>
 __global__ void __launch_bounds__(EpiCfg<MODE>::threads, 1)
 gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                const GemmParams p)
+                const std::conditional_t<QOUT, GemmParamsQ, GemmParams> p)
 {
     using E = EpiCfg<MODE>;
+    static_assert(!QOUT || E::cols == 128, "fused output quantization needs one 1x128 group per thread");
     constexpr int kEpiWarps = E::warps;
     constexpr int kColsPerThread = E::cols;
     constexpr int kChunks = E::chunks;
@@ -457,6 +473,63 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             // ---- store the tile: row m, this thread's kColsPerThread columns
             const int64_t m = (int64_t)tm * kBM + row_in_tile;
             const int n_base = tn * kBN + col0;
+            if constexpr (QOUT) {
+                const int valid = p.N - n_base;            // columns of this group below N
+                if (m < p.M && valid > 0) {
+                    // 1. round to bf16 (the output's values) and store them if wanted
+                    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + m * p.ldd;
+#pragma unroll
+                    for (int j = 0; j < kColsPerThread / 8; ++j) {
+                        const int n = n_base + 8 * j;
+                        const uint32_t ww[4] = {cvt_bf16x2(acc[4 * j].x, acc[4 * j].y),
+                                                cvt_bf16x2(acc[4 * j + 1].x, acc[4 * j + 1].y),
+                                                cvt_bf16x2(acc[4 * j + 2].x, acc[4 * j + 2].y),
+                                                cvt_bf16x2(acc[4 * j + 3].x, acc[4 * j + 3].y)};
+                        if (p.D != nullptr) {
+                            if (p.vec_out && n + 8 <= p.N) {
+                                *reinterpret_cast<uint4*>(dst + n) = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+                            } else if (n < p.N) {
+                                uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
+                                for (int t = 0; t < min(8, p.N - n); ++t)
+                                    d16[n + t] = (uint16_t)((ww[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+                            }
+                        }
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            acc[4 * j + t] = make_float2(__uint_as_float(ww[t] << 16), __uint_as_float(ww[t] & 0xFFFF0000u));
+                    }
+                    // 2. the group's amax over its valid columns, scale, bytes
+                    float amax = 0.f;
+#pragma unroll
+                    for (int j = 0; j < kColsPerThread / 2; ++j) {
+                        if (2 * j < valid) amax = fmaxf(amax, fabsf(acc[j].x));
+                        if (2 * j + 1 < valid) amax = fmaxf(amax, fabsf(acc[j].y));
+                    }
+                    const float sc = scale_from_amax(amax);
+                    uint8_t* qrow = p.qout + m * p.ldq_out + n_base;
+#pragma unroll
+                    for (int j = 0; j < kColsPerThread / 16; ++j) {
+                        float f0[8], f1[8];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            f0[2 * t] = acc[8 * j + t].x;
+                            f0[2 * t + 1] = acc[8 * j + t].y;
+                            f1[2 * t] = acc[8 * j + 4 + t].x;
+                            f1[2 * t + 1] = acc[8 * j + 4 + t].y;
+                        }
+                        const uint2 lo = quant8(f0, sc), hi = quant8(f1, sc);
+                        if (16 * j + 16 <= valid) {
+                            *reinterpret_cast<uint4*>(qrow + 16 * j) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+                        } else if (16 * j < valid) {
+                            const uint32_t bw[4] = {lo.x, lo.y, hi.x, hi.y};
+                            for (int t = 0; t < valid - 16 * j; ++t)
+                                qrow[16 * j + t] = (uint8_t)((bw[t >> 2] >> ((t & 3) * 8)) & 0xFFu);
+                        }
+                    }
+                    p.sout[m + (int64_t)(n_base / 128) * p.lds_out] = __frcp_rn(sc);
+                }
+                continue;
+            }
             if (m < p.M) {
                 if (p.splits > 1) {
                     float* dst = p.ws + ((int64_t)split * p.M + m) * p.ldw;

@@ -58,11 +58,14 @@ def lib():
         L.fp8_scaled_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
         L.fp8_scaled_gemm_workspace_size.restype = sz
         L.fp8_scaled_gemm.argtypes = [i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, i32, p, i64, i32, p, sz, p]
+        L.fp8_scaled_gemm_quant.argtypes = [i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, i32, p, i64,
+                                            p, i64, p, i64, p]
         L.fp8bs_status_string.argtypes = [i32]
         L.fp8bs_status_string.restype = ctypes.c_char_p
         L.fp8bs_check_device_error.argtypes = [p]
         for fn in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_tensor",
-                   "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8bs_check_device_error"):
+                   "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_quant",
+                   "fp8bs_check_device_error"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -239,6 +242,39 @@ def fp8_scaled_gemm(A: torch.Tensor, Bt: torch.Tensor, scale_a: torch.Tensor, sc
                                                     SCALE_COL_MAJOR, out.data_ptr(), _ld(out), oc, wp, wn,
                                                     _stream(A)))
     return out
+
+
+def fp8_scaled_gemm_quant(A: torch.Tensor, Bt: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor, mode: int,
+                          out: Optional[torch.Tensor] = None, store_out: bool = True,
+                          q_out: Optional[torch.Tensor] = None, scale_out: Optional[torch.Tensor] = None):
+    """D = scaled(A . Bt^T) in bf16, quantized 1x128 along N in the GEMM's
+    epilogue: returns (D or None, q uint8 M x N, scale_inv grid M x ceil(N/128)),
+    byte-identical to fp8_quant_1x128(D).  store_out=False skips writing D."""
+    M, K = A.shape
+    N, K2 = Bt.shape
+    if K2 != K:
+        raise ValueError("A and Bt must share K")
+    if store_out and out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    if not store_out:
+        out = None
+    if q_out is None:
+        # the byte rows start 16-byte aligned (pitch rounded up to 16)
+        q_out = torch.empty((M, (N + 15) // 16 * 16), dtype=torch.uint8, device=A.device)[:, :N]
+    if scale_out is None:
+        scale_out = colmajor_grid(M, (N + 127) // 128, A.device)
+    if mode == SCALE_BLOCK_1x128_128x128:
+        ld_sa = _grid_ld(scale_a, M)
+        ld_sb = _grid_ld(scale_b, scale_b.shape[0])
+    else:
+        ld_sa = ld_sb = 0
+    dp, ldd = (out.data_ptr(), _ld(out)) if out is not None else (0, 0)
+    _check("fp8_scaled_gemm_quant",
+           lib().fp8_scaled_gemm_quant(M, N, K, A.data_ptr(), _ld(A), Bt.data_ptr(), _ld(Bt), scale_a.data_ptr(),
+                                       ld_sa, scale_b.data_ptr(), ld_sb, mode, SCALE_COL_MAJOR, dp, ldd,
+                                       q_out.data_ptr(), q_out.stride(0), scale_out.data_ptr(),
+                                       _grid_ld(scale_out, M), _stream(A)))
+    return out, q_out, scale_out
 
 
 def fp8bs_status_string(status: int) -> str:

@@ -9,6 +9,9 @@ only the named kernel runs R times):
   gemm_dgrad   Llama4 dgrad GEMM 16640 x 8192 x 5120 (dy . W), 1x128 x 128x128, bf16 out
   gemm_tensor  16640 x 5120 x 8192 per-tensor scales, bf16 out
   gemm_rowwise 16640 x 5120 x 8192 rowwise scales, bf16 out
+  gemm_fwd_quant       the forward GEMM with its output quantized 1x128 in the epilogue (bf16 out stored)
+  gemm_fwd_quant_only  the same without storing the bf16 output
+  gemm_fwd_then_quant  the forward GEMM, then fp8_quant_1x128 of its output (two launches)
   gemm_longk   256 x 512 x 128128 (k_blocks 1001), 1x128 x 128x128, split-K, bf16 out
   quant_rows   1x128 quantization of a 32768 x 32768 bf16 matrix
   quant_cols   1x128 along rows (transposed output) of a 16640 x 8192 bf16 matrix
@@ -98,6 +101,27 @@ def _gemm_case(name):
     return (lambda: ops.fp8_scaled_gemm(qa, qb, sa, sb, mode, out=out, workspace=wsb)), flops, "TFLOP/s"
 
 
+def _fused_case(name):
+    x, W, _ = inputs.llama4(5120, 8192)
+    qa, sa = ops.fp8_quant_1x128(x.cuda())
+    qb, sb, _, _ = ops.fp8_quant_128x128(W.cuda())
+    mode = ops.SCALE_BLOCK_1x128_128x128
+    M = inputs.LLAMA4_M
+    y = torch.empty((M, 5120), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((M, 5120), dtype=torch.uint8, device="cuda")
+    s = ops.colmajor_grid(M, 40, "cuda")
+    flops = 2.0 * M * 5120 * 8192
+    if name == "gemm_fwd_then_quant":
+        def fn():
+            ops.fp8_scaled_gemm(qa, qb, sa, sb, mode, out=y)
+            ops.fp8_quant_1x128(y, q=q, scale_inv=s)
+    else:
+        store = name == "gemm_fwd_quant"
+        fn = lambda: ops.fp8_scaled_gemm_quant(qa, qb, sa, sb, mode, out=y, store_out=store, q_out=q, scale_out=s)
+    torch.cuda.synchronize()
+    return fn, flops, "TFLOP/s"
+
+
 def _quant_case(name):
     parts = name.split("_")
     if len(parts) == 3 and parts[2].isdigit():
@@ -139,13 +163,20 @@ def _quant_case(name):
 
 
 CONFIG_CASES = (["gemm_tiny", "gemm_pertensor_small", "gemm_rowwise_small", "gemm_fwd", "gemm_dgrad",
-                 "gemm_wgrad", "gemm_tensor", "gemm_rowwise", "gemm_longk", "quant_dual"]
+                 "gemm_wgrad", "gemm_tensor", "gemm_rowwise", "gemm_longk", "gemm_fwd_then_quant",
+                 "gemm_fwd_quant", "gemm_fwd_quant_only", "quant_dual"]
                 + [f"quant_rows_{n}" for n in inputs.QUANT_SWEEP_SIZES]
                 + [f"quant_tile_{n}" for n in inputs.QUANT_SWEEP_SIZES])
 
 
+def _case(name):
+    if name in ("gemm_fwd_quant", "gemm_fwd_quant_only", "gemm_fwd_then_quant"):
+        return _fused_case(name)
+    return _gemm_case(name) if name.startswith("gemm") else _quant_case(name)
+
+
 def _time(case, reps):
-    fn, work, unit = _gemm_case(case) if case.startswith("gemm") else _quant_case(case)
+    fn, work, unit = _case(case)
     fn()
     torch.cuda.synchronize()
     rounds = []
@@ -181,10 +212,7 @@ def main(argv=None):
     a = ap.parse_args(argv)
     if a.case == "configs":
         return configs(a.reps)
-    if a.case.startswith("gemm"):
-        fn, work, unit = _gemm_case(a.case)
-    else:
-        fn, work, unit = _quant_case(a.case)
+    fn, work, unit = _case(a.case)
     fn()
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * a.reps)]

@@ -257,6 +257,37 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K,
                              void* D, int64_t ldd, fp8bs_dtype out_dtype,
                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * fp8_scaled_gemm_quant -- the scaled GEMM with its bf16 output quantized
+ * 1x128 along N in the epilogue, for a consumer that needs the output in FP8
+ * (the next layer's GEMM), so that the output is not read back from memory
+ * to be quantized.
+ *
+ * Defined by: fp8_scaled_gemm followed by fp8_quant_1x128 on its bf16 output;
+ * pytorch/ao PR #2785 "integrate torch._scaled_mm into Float8BlockwiseLinear
+ * and add bench script" (Benchmarks: the quantization launches are the gap to
+ * the bf16 linear).  The quantized bytes and scales are identical to those of
+ * fp8_quant_1x128 applied to D (the epilogue rounds to bf16 first and applies
+ * the same group rule to the rounded values).
+ *
+ * Arguments as fp8_scaled_gemm (output dtype bf16, no split-K workspace), plus:
+ * D          optional (NULL: the bf16 output is not stored; its quantization is
+ *            still that of the values D would hold), leading dim ldd >= N.
+ * q_out      M x N e4m3 bytes, leading dim ldq_out >= N, ldq_out % 16 == 0.
+ * scale_out  grid M x ceil(N/128) of reciprocal scales, scale_out[m + g*ld_scale_out],
+ *            ld_scale_out >= M, ld_scale_out % 4 == 0.
+ * q_out and scale_out 16-byte aligned.  The caller owns every buffer.
+ * Recipes: TENSOR, ROWWISE and BLOCK_1x128_128x128; BLOCK_1x128_1x128 returns
+ * FP8BS_ERR_UNSUPPORTED.  Errors as fp8_scaled_gemm; nothing is launched when
+ * a check fails.  Asynchronous on `stream`.
+ */
+fp8bs_status fp8_scaled_gemm_quant(int64_t M, int64_t N, int64_t K,
+                                   const uint8_t* A, int64_t lda, const uint8_t* Bt, int64_t ldb,
+                                   const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
+                                   fp8bs_scale_mode mode, fp8bs_scale_layout layout,
+                                   void* D, int64_t ldd, uint8_t* q_out, int64_t ldq_out,
+                                   float* scale_out, int64_t ld_scale_out, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* fp8bs_status_string(fp8bs_status s);
 

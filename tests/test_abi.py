@@ -33,7 +33,8 @@ def L():
 def test_header_declares_the_path(L):
     names = declared_functions()
     for want in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_tensor",
-                 "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_workspace_size", "fp8bs_status_string",
+                 "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_quant", "fp8_scaled_gemm_workspace_size",
+                 "fp8bs_status_string",
                  "fp8bs_check_device_error", "fp8_quant_tensor_workspace_size"):
         assert want in names
 
@@ -138,3 +139,24 @@ def test_workspace_size_is_zero_for_large_problems(L):
     assert L.fp8_scaled_gemm_workspace_size(16640, 5120, 8192, 2) == 0
     small = L.fp8_scaled_gemm_workspace_size(256, 512, 128000, 2)
     assert small > 0 and small % 16 == 0
+
+
+def gq(L, M=256, N=384, K=256, A=GOOD, lda=256, B=GOOD, ldb=256, sa=GOOD, lsa=256, sb=GOOD, lsb=4, mode=2, lay=0,
+       D=GOOD, ldd=384, q=GOOD, ldq=384, s=GOOD, lds=256):
+    return L.fp8_scaled_gemm_quant(M, N, K, A, lda, B, ldb, sa, lsa, sb, lsb, mode, lay, D, ldd, q, ldq, s, lds, None)
+
+
+def test_gemm_quant_validation(L):
+    assert gq(L, q=0) == INVALID                    # no quantized output
+    assert gq(L, s=0) == INVALID                    # no scales
+    assert gq(L, ldq=256) == INVALID                # ldq_out < N
+    assert gq(L, lds=128) == INVALID                # ld_scale_out < M
+    assert gq(L, q=BAD) == ALIGN
+    assert gq(L, s=GOOD + 8) == ALIGN
+    assert gq(L, ldq=392) == ALIGN                  # ldq_out % 16
+    assert gq(L, lds=258) == ALIGN                  # ld_scale_out % 4
+    assert gq(L, mode=3, lsb=384) == UNSUPPORTED    # 1x128 x 1x128: 64 columns per promotion thread
+    assert gq(L, mode=7) == UNSUPPORTED
+    assert gq(L, A=0) == INVALID
+    assert gq(L, D=GOOD, ldd=100) == INVALID        # stored output with ldd < N
+

@@ -351,3 +351,35 @@ def test_long_k_fp32_output(recipe):
     qao, sao = oracle.quant_1x128(bits(goT), rows=rows)
     assert_f32_close(D[torch.as_tensor(rows, device="cuda")], oracle.gemm(qao, qbo, sao, sbo, mode),
                      f"long K fp32 out {recipe}")
+
+
+@pytest.mark.parametrize("mode", [ops.SCALE_TENSOR, ops.SCALE_ROWWISE, ops.SCALE_BLOCK_1x128_128x128])
+@pytest.mark.parametrize("M,N,K", [(300, 264, 1024), (256, 1008, 640), (1280, 2056, 512)])
+def test_gemm_quant_output(M, N, K, mode):
+    """The GEMM with its bf16 output quantized 1x128 along N in the epilogue:
+    D within the bf16 tolerance of the oracle, and the quantized bytes and
+    scales bit-exact against the oracle's 1x128 quantization of the GPU's own D
+    (N not a multiple of 128: a ragged last group; more tiles than SMs).  The
+    same call without storing D gives the same bytes and scales."""
+    rng = np.random.default_rng(M + N + K)
+    A = inputs.random_e4m3_bytes(M, K, seed=M)
+    B = inputs.random_e4m3_bytes(N, K, seed=N)
+    sa, sb = make_scales(rng, mode, M, N, K)
+    Ad, Bd, sad, sbd = A.cuda(), B.cuda(), to_gpu_scales(sa, mode), to_gpu_scales(sb, mode)
+    D, q, s = ops.fp8_scaled_gemm_quant(Ad, Bd, sad, sbd, mode)
+    D2, q2, s2 = ops.fp8_scaled_gemm_quant(Ad, Bd, sad, sbd, mode, store_out=False)
+    torch.cuda.synchronize()
+    no_device_error()
+    assert D2 is None
+    assert_bf16_close(D, oracle.gemm(A.numpy(), B.numpy(), sa, sb, mode), f"D M{M} N{N} K{K}")
+    qo, so = oracle.quant_1x128(bits(D.cpu()))
+    assert_bytes_equal(q, qo, "quantized output")
+    assert_scales_equal(grid_np(s), so, "output scales")
+    assert torch.equal(q, q2)
+    assert_scales_equal(grid_np(s2), so, "output scales without D")
+    if N % 16 == 0:
+        # and equal to the separate quantization launch on D (which needs N % 16 == 0)
+        q3, s3 = ops.fp8_quant_1x128(D)
+        torch.cuda.synchronize()
+        assert torch.equal(q, q3)
+        assert_scales_equal(grid_np(s), grid_np(s3), "vs fp8_quant_1x128(D)")
