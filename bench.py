@@ -40,9 +40,8 @@ FP8_SPEC_TFLOPS = 4500.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
 # GEMM launch of the (5120, 8192) layer (16640 x 5120 x 8192), from an ncu
-# capture, keyed by a hash of the kernel source it was taken on (the summary is
-# profiles/gemm_fp8_fwd_llama4.md).  A changed kernel reports null until it is
-# captured again.
+# capture, keyed by a hash of the kernel source it was taken on.  A changed
+# kernel reports null until it is captured again.
 GEMM_TRAFFIC = {"1e8ca1a0fe545570": 572.1e6}
 
 

@@ -657,8 +657,7 @@ extern "C" fp8bs_status fp8bs_selftest_wait_timeout(uint64_t limit_ns, cudaStrea
 
 namespace {
 constexpr int kNoAllocPartials = 4096;                  // floats of scratch (16 KB)
-constexpr int64_t kNoAllocElemsPerPartial = 65536;      // elements reduced per amax CTA
-constexpr int64_t kNoAllocMaxElems = (int64_t)kNoAllocPartials * kNoAllocElemsPerPartial;
+constexpr int64_t kNoAllocMaxElems = int64_t(1) << 28;  // the documented size limit
 std::atomic<float*> g_noalloc_scratch[kMaxDevices]{};   // device address of the array, per device
 std::mutex g_noalloc_mutex;
 }  // namespace
@@ -692,10 +691,12 @@ extern "C" fp8bs_status fp8_quant_tensor_noalloc(const void* x, fp8bs_dtype xt, 
             g_noalloc_scratch[dev].store(partial, std::memory_order_release);
         }
     }
-    // every partial slot the second kernel reads is written by the first one in
-    // this same call, so nothing left by an earlier call needs clearing
-    const int parts = (int)std::max<int64_t>(1, cdiv(n, kNoAllocElemsPerPartial));
-    if (parts > kNoAllocPartials) return FP8BS_ERR_WORKSPACE;
+    // One amax partial per 8192 elements (as fp8_quant_tensor partitions the
+    // tensor), at most one per scratch slot: the amax kernel's grid-stride loop
+    // covers any n with any grid.  Every partial slot the second kernel reads is
+    // written by the first one in this same call, so nothing left by an earlier
+    // call needs clearing.
+    const int parts = (int)std::max<int64_t>(1, std::min<int64_t>(kNoAllocPartials, cdiv(n, 8192)));
     const int64_t chunks = n / 8;
     if (xt == FP8BS_BF16) {
         tensor_amax_kernel<__nv_bfloat16><<<parts, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), n, partial);

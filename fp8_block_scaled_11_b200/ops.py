@@ -63,9 +63,10 @@ def lib():
         L.fp8bs_status_string.argtypes = [i32]
         L.fp8bs_status_string.restype = ctypes.c_char_p
         L.fp8bs_check_device_error.argtypes = [p]
+        L.fp8_quant_tensor_noalloc.argtypes = [p, i32, i64, p, p, p]
         for fn in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_tensor",
                    "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_quant",
-                   "fp8bs_check_device_error"):
+                   "fp8bs_check_device_error", "fp8_quant_tensor_noalloc"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -290,15 +291,28 @@ def fp8_quant_tensor_noalloc(x: torch.Tensor, q: Optional[torch.Tensor] = None,
                              scale_inv: Optional[torch.Tensor] = None):
     """Per-tensor quantization through fp8_quant_tensor_noalloc (no workspace:
     the library uses its built-in 16 KB scratch).  Returns (q, scale_inv[1]);
-    pass preallocated q / scale_inv to keep the call itself allocation-free."""
-    L = lib()
-    fn = L.fp8_quant_tensor_noalloc
-    fn.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
-    fn.restype = ctypes.c_int
+    pass preallocated q / scale_inv to keep the call itself allocation-free.
+
+    The call cannot copy (a copy would allocate), so x must already be a
+    contiguous bf16 / fp32 tensor on the current CUDA device; q must be a
+    contiguous uint8 tensor with as many elements as x and scale_inv a
+    contiguous fp32 tensor with at least one element, on the same device.
+    Anything else raises ValueError before the library is called."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if x.device != dev or not x.is_contiguous():
+        raise ValueError("fp8_quant_tensor_noalloc: x must be contiguous and on the current CUDA device")
+    xt = _dtype_code(x)
     if q is None:
         q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scale_inv is None:
         scale_inv = torch.empty((1,), dtype=torch.float32, device=x.device)
-    _check("fp8_quant_tensor_noalloc", fn(x.data_ptr(), _dtype_code(x), x.numel(), q.data_ptr(),
-                                          scale_inv.data_ptr(), _stream(x)))
+    if q.dtype != torch.uint8 or q.numel() != x.numel() or not q.is_contiguous() or q.device != dev:
+        raise ValueError("fp8_quant_tensor_noalloc: q must be a contiguous uint8 tensor of x.numel() elements "
+                         "on the current CUDA device")
+    if (scale_inv.dtype != torch.float32 or scale_inv.numel() < 1 or not scale_inv.is_contiguous()
+            or scale_inv.device != dev):
+        raise ValueError("fp8_quant_tensor_noalloc: scale_inv must be a contiguous fp32 tensor with at least "
+                         "one element on the current CUDA device")
+    _check("fp8_quant_tensor_noalloc", lib().fp8_quant_tensor_noalloc(x.data_ptr(), xt, x.numel(), q.data_ptr(),
+                                                                      scale_inv.data_ptr(), _stream(x)))
     return q, scale_inv

@@ -17,8 +17,10 @@
  *
  * Conventions for every entry point:
  *   - All pointers are DEVICE pointers owned by the caller.  The library
- *     allocates no device memory and keeps no device state except one int of
- *     device-side error flag (see fp8bs_check_device_error).
+ *     allocates no device memory.  Its only device state is compiled in: one
+ *     int of device-side error flag (see fp8bs_check_device_error) and the
+ *     16 KB scratch array of fp8_quant_tensor_noalloc, both held by every GPU
+ *     that loads the library until the process exits.
  *   - Every call is asynchronous on `stream` (0 = legacy default stream) and
  *     never synchronizes, except fp8bs_check_device_error.
  *   - Arguments are validated before anything is launched; on an error status

@@ -1,6 +1,6 @@
 """Single-kernel cases for profiling (ncu) and per-kernel timing.
 
-  python -m fp8_block_scaled_11_b200.profile_cases <case> [--reps R] [--time]
+  python profile_cases.py <case> [--reps R] [--time]
 
 Cases (seeded inputs of the workloads, operands prepared before the loop so
 only the named kernel runs R times):
@@ -23,7 +23,7 @@ only the named kernel runs R times):
   quant_rows_<n>, quant_tile_<n>   the quantization sweep at n x n bf16 (n = 1024 ... 32768)
 With --time, each launch is timed with CUDA events and the mean is printed.
 
-  python -m fp8_block_scaled_11_b200.profile_cases configs [--reps R]
+  python profile_cases.py configs [--reps R]
 
 times every case above (the median of three rounds of R timed launches each)
 and prints one table.
@@ -35,7 +35,7 @@ import sys
 
 import torch
 
-from . import inputs, ops
+from fp8_block_scaled_11_b200 import inputs, ops
 
 
 def _gemm_case(name):
