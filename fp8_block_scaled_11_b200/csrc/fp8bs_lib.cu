@@ -1,7 +1,9 @@
 // fp8bs_lib.cu -- the C ABI declared in include/fp8bs.h: argument validation,
 // TMA tensor-map encoding, launch configuration, and the device error flag.
 // The kernels are in quant_kernels.cuh and gemm_kernel.cuh (one translation
-// unit, so the error flag is a plain __device__ variable).
+// unit, so the error flag is a plain __device__ variable).  The plain GEMM runs
+// on CTA pairs (gemm_pair_kernel.cuh); the GEMM with its output quantized in
+// the epilogue runs on single CTAs (gemm_kernel.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -15,6 +17,7 @@
 #include "fp8bs.h"
 #include "quant_kernels.cuh"
 #include "gemm_kernel.cuh"
+#include "gemm_pair_kernel.cuh"
 #include "splitk_reduce.cuh"
 
 using namespace fp8bs;
@@ -37,6 +40,7 @@ struct DeviceInfo {
     std::atomic<int> quant_blocks[10]{};     // resident CTAs per SM, per quant kernel kind
     std::atomic<bool> tile_attr_set[8]{};
     std::atomic<int> tile_blocks[8]{};
+    std::atomic<int> pair_clusters[8]{};     // co-resident CTA pairs, per pair-kernel instantiation
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -169,6 +173,39 @@ SplitPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms)
     return s;
 }
 
+// Pair kernel: 256 x 128 output tiles; split-K when the tiles cannot keep half
+// the CTA pairs busy (same rule as plan_gemm, over pairs instead of SMs).
+SplitPlan plan_pair(int64_t M, int64_t N, int64_t K, int num_sms)
+{
+    SplitPlan s;
+    s.tiles_m = (int)cdiv(M, kPairM);
+    s.tiles_n = (int)cdiv(N, kPairN);
+    const int64_t tiles = (int64_t)s.tiles_m * s.tiles_n;
+    const int64_t Kb = cdiv(K, kBK);
+    const int pairs = std::max(1, num_sms / 2);
+    int splits = 1;
+    if (tiles * 2 <= pairs) {
+        splits = (int)std::min<int64_t>(pairs / tiles, std::max<int64_t>(1, Kb / 8));
+        splits = std::max(1, std::min(splits, 64));
+    }
+    s.splits = splits;
+    s.ldw = (N + 3) & ~int64_t(3);
+    s.ws_bytes = splits > 1 ? (size_t)splits * (size_t)M * (size_t)s.ldw * sizeof(float) : 0;
+    return s;
+}
+
+// Which GEMM kernel a call runs: the CTA-pair kernel for an MN-major B (the
+// single-CTA kernel reads K-major operands only) and for outputs too small to
+// fill the GPU without splitting K (fewer, wider splits: the long-K case), the
+// single-CTA kernel otherwise (faster on large outputs, where its two 256-column
+// accumulators are fed by a single TMA ring) and for the fused output quantization.
+bool use_pair(int64_t M, int64_t N, int64_t K, bool b_mn, bool quant_out, int num_sms)
+{
+    if (quant_out) return false;
+    if (b_mn) return true;
+    return plan_pair(M, N, K, num_sms).splits > 1;
+}
+
 int num_sms_current()
 {
     DeviceInfo* d = nullptr;
@@ -202,6 +239,45 @@ fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap
     }
     const int grid = (int)std::min<int64_t>(p.num_units, d->num_sms);
     k<<<grid, EpiCfg<MODE>::threads, SmemLayout::alloc, stream>>>(tA, tB, tSA, tSB, p);
+    return launch_status();
+}
+
+// Launch of the pair kernel: clusters of two CTAs, one pair per two SMs (as
+// many as can be co-resident), persistent over the units.
+template <int MODE, bool BMN>
+fp8bs_status launch_pair(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA,
+                         const CUtensorMap& tSB, const GemmParams& p, cudaStream_t stream)
+{
+    auto k = gemm_fp8_pair_kernel<MODE, BMN>;
+    constexpr int slot = MODE + (BMN ? 4 : 0);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
+    cfg.dynamicSmemBytes = PairSmem::alloc;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nc = d->pair_clusters[slot].load(std::memory_order_acquire);
+    if (nc == 0) {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        nc = d->pair_clusters[slot].load(std::memory_order_relaxed);
+        if (nc == 0) {
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PairSmem::alloc) !=
+                cudaSuccess)
+                return FP8BS_ERR_CUDA;
+            cfg.gridDim = dim3(2 * std::max(1, d->num_sms / 2), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&nc, k, &cfg) != cudaSuccess) return FP8BS_ERR_CUDA;
+            if (nc < 1) return FP8BS_ERR_UNSUPPORTED;
+            d->pair_clusters[slot].store(nc, std::memory_order_release);
+        }
+    }
+    const int64_t clusters = std::min<int64_t>(p.num_units, nc);
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, k, tA, tB, tSA, tSB, p) != cudaSuccess) return FP8BS_ERR_CUDA;
     return launch_status();
 }
 
@@ -451,7 +527,11 @@ size_t fp8_scaled_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8bs_sca
 {
     (void)mode;
     if (M < 1 || N < 1 || K < 1) return 0;
-    return plan_gemm(M, N, K, num_sms_current()).ws_bytes;
+    const int sms = num_sms_current();
+    // the larger of the two kernels' needs: fp8_scaled_gemm_ex with an
+    // MN-major B always runs the pair kernel
+    return std::max(plan_pair(M, N, K, sms).ws_bytes,
+                    use_pair(M, N, K, false, false, sms) ? size_t(0) : plan_gemm(M, N, K, sms).ws_bytes);
 }
 
 }  // extern "C"
@@ -466,9 +546,9 @@ struct QuantOut {
     int64_t lds = 0;
 };
 
-fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* Bt,
-                         int64_t ldb, const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
-                         fp8bs_scale_mode mode, fp8bs_scale_layout layout, void* D, int64_t ldd,
+fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* B,
+                         int64_t ldb, bool b_mn, const float* scale_a, int64_t ld_sa, const float* scale_b,
+                         int64_t ld_sb, fp8bs_scale_mode mode, fp8bs_scale_layout layout, void* D, int64_t ldd,
                          fp8bs_dtype out_dtype, void* workspace, size_t workspace_bytes, const QuantOut& qo,
                          cudaStream_t stream)
 {
@@ -476,11 +556,12 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
     if (mode < FP8BS_SCALE_TENSOR || mode > FP8BS_SCALE_BLOCK_1x128_1x128) return FP8BS_ERR_UNSUPPORTED;
     if (layout != FP8BS_SCALE_COL_MAJOR || !valid_dtype(out_dtype)) return FP8BS_ERR_UNSUPPORTED;
     if (quant_out && (mode == FP8BS_SCALE_BLOCK_1x128_1x128 || out_dtype != FP8BS_BF16)) return FP8BS_ERR_UNSUPPORTED;
-    if (A == nullptr || Bt == nullptr || scale_a == nullptr || scale_b == nullptr) return FP8BS_ERR_INVALID_ARG;
+    if (b_mn && (quant_out || mode == FP8BS_SCALE_BLOCK_1x128_1x128)) return FP8BS_ERR_UNSUPPORTED;
+    if (A == nullptr || B == nullptr || scale_a == nullptr || scale_b == nullptr) return FP8BS_ERR_INVALID_ARG;
     if (D == nullptr && !quant_out) return FP8BS_ERR_INVALID_ARG;
     if (M < 1 || N < 1 || K < 16) return FP8BS_ERR_INVALID_ARG;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8BS_ERR_INVALID_ARG;
-    if (lda < K || ldb < K || (D != nullptr && ldd < N)) return FP8BS_ERR_INVALID_ARG;
+    if (lda < K || ldb < (b_mn ? N : K) || (D != nullptr && ldd < N)) return FP8BS_ERR_INVALID_ARG;
     if (quant_out) {
         if (qo.s == nullptr || qo.ldq < N || qo.lds < M) return FP8BS_ERR_INVALID_ARG;
         if (!aligned16(qo.q) || !aligned16(qo.s) || qo.ldq % 16 || qo.lds % 4) return FP8BS_ERR_ALIGNMENT;
@@ -489,19 +570,21 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
     const bool block = (mode == FP8BS_SCALE_BLOCK_1x128_128x128 || mode == FP8BS_SCALE_BLOCK_1x128_1x128);
     if (block) {
         if (ld_sa < M) return FP8BS_ERR_INVALID_ARG;
-        if (mode == FP8BS_SCALE_BLOCK_1x128_128x128 && ld_sb < Nb) return FP8BS_ERR_INVALID_ARG;
+        if (mode == FP8BS_SCALE_BLOCK_1x128_128x128 && ld_sb < (b_mn ? Kb : Nb)) return FP8BS_ERR_INVALID_ARG;
         if (mode == FP8BS_SCALE_BLOCK_1x128_1x128 && ld_sb < N) return FP8BS_ERR_INVALID_ARG;
         if (ld_sa % 4 || ld_sb % 4) return FP8BS_ERR_ALIGNMENT;
     }
     if (K % 16 || lda % 16 || ldb % 16) return FP8BS_ERR_ALIGNMENT;
-    if (!aligned16(A) || !aligned16(Bt) || !aligned16(scale_a) || !aligned16(scale_b)) return FP8BS_ERR_ALIGNMENT;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(scale_a) || !aligned16(scale_b)) return FP8BS_ERR_ALIGNMENT;
     if (reinterpret_cast<uintptr_t>(D) % dtype_size(out_dtype)) return FP8BS_ERR_ALIGNMENT;
     const int vec_out = D != nullptr && aligned16(D) && (ldd * (int64_t)dtype_size(out_dtype)) % 16 == 0;
     DeviceInfo* d = nullptr;
     fp8bs_status st = get_device(&d);
     if (st != FP8BS_OK) return st;
 
-    SplitPlan plan = plan_gemm(M, N, K, d->num_sms);
+    // single-CTA tiles (128 x 256) or CTA pairs (256 x 128)
+    const bool pair = use_pair(M, N, K, b_mn, quant_out, d->num_sms);
+    SplitPlan plan = pair ? plan_pair(M, N, K, d->num_sms) : plan_gemm(M, N, K, d->num_sms);
     if (quant_out) plan.splits = 1;              // the epilogue quantizes whole tiles
     if (plan.splits > 1) {
         if (workspace == nullptr && workspace_bytes == 0) {
@@ -513,26 +596,47 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
         }
     }
 
+    // operand maps: A rows x 128-byte K slices; B^T likewise (K-major), or B
+    // as the 256 K-rows of a pair-kernel step x 64-byte column slices (MN-major)
+    const uint32_t a_rows = pair ? kCtaM : kBM;
+    const uint32_t bt_rows = pair ? kCtaN : kBN;
     CUtensorMap tA, tB, tSA, tSB;
     std::memset(&tSA, 0, sizeof tSA);
     std::memset(&tSB, 0, sizeof tSB);
-    if ((st = make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, lda, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
+    if ((st = make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, lda, kBK, a_rows, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
         return st;
-    if ((st = make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Bt, K, N, ldb, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
+    if (b_mn) {
+        if ((st = make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, N, K, ldb, kCtaN, kStepKb * kBK, CU_TENSOR_MAP_SWIZZLE_64B)) != FP8BS_OK)
+            return st;
+    } else if ((st = make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, ldb, kBK, bt_rows, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK) {
         return st;
+    }
     const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const uint32_t sa_box = pair ? 128 : kBM;
+    const uint32_t sb_box = pair ? 128 : kBN;
     switch (mode) {
     case FP8BS_SCALE_TENSOR:
         break;
     case FP8BS_SCALE_ROWWISE:
-        if ((st = make_map(&tSA, f32, 4, scale_a, M, 1, (M * 4 + 15) & ~int64_t(15), kBM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
-        if ((st = make_map(&tSB, f32, 4, scale_b, N, 1, (N * 4 + 15) & ~int64_t(15), kBN, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        if ((st = make_map(&tSA, f32, 4, scale_a, M, 1, (M * 4 + 15) & ~int64_t(15), sa_box, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        if ((st = make_map(&tSB, f32, 4, scale_b, N, 1, (N * 4 + 15) & ~int64_t(15), sb_box, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
         break;
-    case FP8BS_SCALE_BLOCK_1x128_128x128:       // scales read directly by the promotion warps
+    case FP8BS_SCALE_BLOCK_1x128_128x128:
+        // single-CTA kernel: the promotion warps read both scales directly;
+        // pair kernel: row scales as for 1x128 x 1x128, the B grid in 16-byte
+        // groups of four blocks ((N-block, K-block), or (K-block, N-block) for MN-major B)
+        if (pair) {
+            if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, sa_box, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+            if (b_mn) {
+                if ((st = make_map(&tSB, f32, 4, scale_b, Kb, Nb, ld_sb * 4, 4, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+            } else if ((st = make_map(&tSB, f32, 4, scale_b, Nb, Kb, ld_sb * 4, 4, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) {
+                return st;
+            }
+        }
         break;
     case FP8BS_SCALE_BLOCK_1x128_1x128:
-        if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, kBM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
-        if ((st = make_map(&tSB, f32, 4, scale_b, N, Kb, ld_sb * 4, kBN, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, sa_box, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        if ((st = make_map(&tSB, f32, 4, scale_b, N, Kb, ld_sb * 4, sb_box, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
         break;
     }
 
@@ -544,7 +648,7 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
     p.tiles_m = plan.tiles_m;
     p.tiles_n = plan.tiles_n;
     p.splits = plan.splits;
-    p.group_m = 16;
+    p.group_m = pair ? 8 : 16;
     p.num_units = (int64_t)plan.tiles_m * plan.tiles_n * plan.splits;
     p.D = D;
     p.ldd = ldd;
@@ -569,12 +673,27 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
         default: return launch_gemm<kModeBlock128, true>(d, tA, tB, tSA, tSB, p, stream);
         }
     }
-    const GemmParams& pb = p;                    // the plain instantiations take the base block
-    switch (mode) {
-    case FP8BS_SCALE_TENSOR: st = launch_gemm<kModeTensor>(d, tA, tB, tSA, tSB, pb, stream); break;
-    case FP8BS_SCALE_ROWWISE: st = launch_gemm<kModeRowwise>(d, tA, tB, tSA, tSB, pb, stream); break;
-    case FP8BS_SCALE_BLOCK_1x128_128x128: st = launch_gemm<kModeBlock128>(d, tA, tB, tSA, tSB, pb, stream); break;
-    case FP8BS_SCALE_BLOCK_1x128_1x128: st = launch_gemm<kModeBlock1x128>(d, tA, tB, tSA, tSB, pb, stream); break;
+    const GemmParams& pb = p;                    // the plain kernels take the base block
+    if (!pair) {
+        switch (mode) {
+        case FP8BS_SCALE_TENSOR: st = launch_gemm<kModeTensor>(d, tA, tB, tSA, tSB, pb, stream); break;
+        case FP8BS_SCALE_ROWWISE: st = launch_gemm<kModeRowwise>(d, tA, tB, tSA, tSB, pb, stream); break;
+        case FP8BS_SCALE_BLOCK_1x128_128x128: st = launch_gemm<kModeBlock128>(d, tA, tB, tSA, tSB, pb, stream); break;
+        case FP8BS_SCALE_BLOCK_1x128_1x128: st = launch_gemm<kModeBlock1x128>(d, tA, tB, tSA, tSB, pb, stream); break;
+        }
+    } else if (b_mn) {
+        switch (mode) {
+        case FP8BS_SCALE_TENSOR: st = launch_pair<kModeTensor, true>(d, tA, tB, tSA, tSB, pb, stream); break;
+        case FP8BS_SCALE_ROWWISE: st = launch_pair<kModeRowwise, true>(d, tA, tB, tSA, tSB, pb, stream); break;
+        default: st = launch_pair<kModeBlock128, true>(d, tA, tB, tSA, tSB, pb, stream); break;
+        }
+    } else {
+        switch (mode) {
+        case FP8BS_SCALE_TENSOR: st = launch_pair<kModeTensor, false>(d, tA, tB, tSA, tSB, pb, stream); break;
+        case FP8BS_SCALE_ROWWISE: st = launch_pair<kModeRowwise, false>(d, tA, tB, tSA, tSB, pb, stream); break;
+        case FP8BS_SCALE_BLOCK_1x128_128x128: st = launch_pair<kModeBlock128, false>(d, tA, tB, tSA, tSB, pb, stream); break;
+        case FP8BS_SCALE_BLOCK_1x128_1x128: st = launch_pair<kModeBlock1x128, false>(d, tA, tB, tSA, tSB, pb, stream); break;
+        }
     }
     if (st != FP8BS_OK) return st;
     if (plan.splits > 1) {
@@ -598,8 +717,20 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, 
                              fp8bs_dtype out_dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream)
 {
     if (D == nullptr) return FP8BS_ERR_INVALID_ARG;
-    return scaled_gemm(M, N, K, A, lda, Bt, ldb, scale_a, ld_sa, scale_b, ld_sb, mode, layout, D, ldd, out_dtype,
-                       workspace, workspace_bytes, QuantOut{}, stream);
+    return scaled_gemm(M, N, K, A, lda, Bt, ldb, false, scale_a, ld_sa, scale_b, ld_sb, mode, layout, D, ldd,
+                       out_dtype, workspace, workspace_bytes, QuantOut{}, stream);
+}
+
+fp8bs_status fp8_scaled_gemm_ex(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* B,
+                                int64_t ldb, fp8bs_major b_major, const float* scale_a, int64_t ld_sa,
+                                const float* scale_b, int64_t ld_sb, fp8bs_scale_mode mode,
+                                fp8bs_scale_layout layout, void* D, int64_t ldd, fp8bs_dtype out_dtype,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (D == nullptr) return FP8BS_ERR_INVALID_ARG;
+    if (b_major != FP8BS_MAJOR_K && b_major != FP8BS_MAJOR_MN) return FP8BS_ERR_UNSUPPORTED;
+    return scaled_gemm(M, N, K, A, lda, B, ldb, b_major == FP8BS_MAJOR_MN, scale_a, ld_sa, scale_b, ld_sb, mode,
+                       layout, D, ldd, out_dtype, workspace, workspace_bytes, QuantOut{}, stream);
 }
 
 fp8bs_status fp8_scaled_gemm_quant(int64_t M, int64_t N, int64_t K, const uint8_t* A, int64_t lda, const uint8_t* Bt,
@@ -614,8 +745,8 @@ fp8bs_status fp8_scaled_gemm_quant(int64_t M, int64_t N, int64_t K, const uint8_
     qo.ldq = ldq_out;
     qo.s = scale_out;
     qo.lds = ld_scale_out;
-    return scaled_gemm(M, N, K, A, lda, Bt, ldb, scale_a, ld_sa, scale_b, ld_sb, mode, layout, D, ldd, FP8BS_BF16,
-                       nullptr, 0, qo, stream);
+    return scaled_gemm(M, N, K, A, lda, Bt, ldb, false, scale_a, ld_sa, scale_b, ld_sb, mode, layout, D, ldd,
+                       FP8BS_BF16, nullptr, 0, qo, stream);
 }
 
 }  // extern "C"

@@ -251,6 +251,131 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N)
          | ((M >> 4) << 24);
 }
 
+
+// ------------------------------------------------------------------ CTA pairs (clusters of two)
+// The two CTAs of a cluster of size 2 form a pair: rank 0 (the leader) issues
+// the pair's tcgen05.mma, which reads A and B from both CTAs' shared memory and
+// writes each CTA's rows of the accumulator into that CTA's TMEM.
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Shared-memory address `addr` of this CTA, as the shared::cluster address of
+// the same offset in the CTA of rank `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (the peer CTA's),
+// with the instruction's default semantics (release at CTA scope): it orders
+// this thread's earlier operations, which is all a TMEM hand-off needs (the
+// tcgen05 loads it follows have completed).  A cluster-scope release would also
+// wait for every earlier memory operation to become visible cluster-wide and
+// measured thousands of cycles per arrival.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Cluster-wide barrier: every thread of every CTA of the cluster executes both.
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 2-D tiled TMA load into this CTA's shared memory whose completion is counted
+// on the mbarrier at `bar_cluster` (a shared::cluster address, which with
+// .cta_group::2 may lie in the peer CTA: both CTAs' loads for one pipeline
+// stage complete on the leader's barrier).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t c0, int32_t c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// TMEM allocation for a CTA pair: the same warp of both CTAs executes it; the
+// same columns are allocated in both CTAs' TMEM.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Pair MMA (issued by one thread of the leader CTA): D[tmem] (+)= A * B^T with
+// M = 256 (128 rows from each CTA's shared memory, each CTA's TMEM receiving its
+// own rows) and B's N columns split in halves between the two CTAs.
+__device__ __forceinline__ void umma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accum)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+
+// Arrives once on the mbarrier at offset `bar` of every CTA in `cta_mask`
+// when all pair MMAs previously issued by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(bar), "h"(cta_mask)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor for an MN-major 8-bit operand tile stored as
+// rows of 64 bytes (64 consecutive MN elements per K index) with the 64-byte
+// swizzle, the layout a TMA load with CU_TENSOR_MAP_SWIZZLE_64B of a 64-byte
+// wide box produces: core groups of 8 K-rows (512 bytes) are `sbo` bytes apart
+// along K; the tile is a single 64-element group along MN, so the leading
+// byte offset is not used.  Descriptor version 1, layout code 4 = 64-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw64(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
+    d |= (uint64_t)1u << 16;                           // leading byte offset (unused)
+    d |= (uint64_t)(512u >> 4) << 32;                  // stride byte offset: 8 K-rows x 64 B
+    d |= (uint64_t)1u << 46;                           // version
+    d |= (uint64_t)4u << 61;                           // SWIZZLE_64B
+    return d;
+}
+
+// Instruction descriptor for kind::f8f6f4 (E4M3 x E4M3 -> F32), A K-major,
+// B K-major (b_mn = 0) or MN-major (b_mn = 1).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32_major(uint32_t M, uint32_t N, uint32_t b_mn)
+{
+    return idesc_e4m3_f32(M, N) | (b_mn << 16);
+}
+
 // ------------------------------------------------------------------ converts
 // Two fp32 -> two e4m3 (round to nearest even, saturate to +-448), packed in
 // 16 bits: `lo` goes to the low byte.

@@ -13,7 +13,9 @@ pytorch/ao PR #4209 (Findings So Far and review thread):
 x: M x K, W: N x K, dy: M x N (all bf16); outputs bf16.  Three quantization
 launches per step -- x in both 1x128 directions from one read, W with its
 transposed copy, dy in both directions from one read -- and three GEMM
-launches.
+launches.  With ``dgrad_wt_copy=False`` W is quantized once and dgrad reads
+the forward's W_q in its stored orientation (B MN-major, fp8_scaled_gemm_ex):
+the same result without the transposed copy, on the CTA-pair GEMM kernel.
 """
 from __future__ import annotations
 
@@ -27,8 +29,9 @@ class Fp8LinearStep:
 
     LAUNCHES_PER_STEP = 6
 
-    def __init__(self, M: int, N: int, K: int, device="cuda"):
+    def __init__(self, M: int, N: int, K: int, device="cuda", dgrad_wt_copy: bool = True):
         self.M, self.N, self.K = M, N, K
+        self.dgrad_wt_copy = dgrad_wt_copy
         d = device
         u8 = torch.uint8
         g = ops.colmajor_grid
@@ -36,7 +39,9 @@ class Fp8LinearStep:
         # forward / dgrad operands
         self.xq, self.xs = torch.empty((M, K), dtype=u8, device=d), g(M, cd(K), d)
         self.wq, self.ws = torch.empty((N, K), dtype=u8, device=d), g(cd(N), cd(K), d)
-        self.wtq, self.wts = torch.empty((K, N), dtype=u8, device=d), g(cd(K), cd(N), d)
+        self.wtq = self.wts = None
+        if dgrad_wt_copy:
+            self.wtq, self.wts = torch.empty((K, N), dtype=u8, device=d), g(cd(K), cd(N), d)
         self.dyq, self.dys = torch.empty((M, N), dtype=u8, device=d), g(M, cd(N), d)
         # wgrad operands (quantized along tokens, stored transposed)
         self.dytq, self.dyts = torch.empty((N, M), dtype=u8, device=d), g(N, cd(M), d)
@@ -53,7 +58,8 @@ class Fp8LinearStep:
 
     def quantize(self, x: torch.Tensor, W: torch.Tensor, dy: torch.Tensor):
         ops.fp8_quant_1x128_dual(x, out=(self.xq, self.xs, self.xtq, self.xts))
-        ops.fp8_quant_128x128(W, want_q=True, want_qt=True, out=(self.wq, self.ws, self.wtq, self.wts))
+        ops.fp8_quant_128x128(W, want_q=True, want_qt=self.dgrad_wt_copy,
+                              out=(self.wq, self.ws, self.wtq, self.wts))
         ops.fp8_quant_1x128_dual(dy, out=(self.dyq, self.dys, self.dytq, self.dyts))
 
     def gemms(self, mark=None):
@@ -64,7 +70,11 @@ class Fp8LinearStep:
         mark(0)
         ops.fp8_scaled_gemm(self.xq, self.wq, self.xs, self.ws, B2, out=self.y, workspace=self.workspace)
         mark(1)
-        ops.fp8_scaled_gemm(self.dyq, self.wtq, self.dys, self.wts, B2, out=self.dx, workspace=self.workspace)
+        if self.dgrad_wt_copy:
+            ops.fp8_scaled_gemm(self.dyq, self.wtq, self.dys, self.wts, B2, out=self.dx, workspace=self.workspace)
+        else:
+            ops.fp8_scaled_gemm_ex(self.dyq, self.wq, ops.MAJOR_MN, self.dys, self.ws, B2, out=self.dx,
+                                   workspace=self.workspace)
         mark(2)
         ops.fp8_scaled_gemm(self.dytq, self.xtq, self.dyts, self.xts, B3, out=self.dW, workspace=self.workspace)
         mark(3)
@@ -83,12 +93,14 @@ class Fp8LinearStep:
 
     def quant_bytes(self) -> float:
         """Algorithmic HBM bytes of the three quantization launches: each bf16
-        input read once (2 B per element), two e4m3 outputs written (2 x 1 B
-        per element), plus 4 bytes per scale written."""
+        input read once (2 B per element), its e4m3 outputs written (1 B per
+        element each: two for x and dy, one for W unless the transposed copy
+        is kept), plus 4 bytes per scale written."""
         M, N, K = self.M, self.N, self.K
         cd = lambda a: (a + 127) // 128
+        copies = 2 if self.dgrad_wt_copy else 1
         b = 0.0
         b += M * K * 4 + 4 * M * cd(K) + 4 * K * cd(M)     # x: 1x128 along K and along tokens
-        b += N * K * 4 + 2 * 4 * cd(N) * cd(K)             # W 128x128 + transposed copy
+        b += N * K * (2 + copies) + copies * 4 * cd(N) * cd(K)   # W 128x128 (+ transposed copy)
         b += M * N * 4 + 4 * M * cd(N) + 4 * N * cd(M)     # dy: 1x128 along N and along tokens
         return b

@@ -29,6 +29,7 @@ STATUS_NAMES = {
 BF16, F32 = 0, 1
 SCALE_TENSOR, SCALE_ROWWISE, SCALE_BLOCK_1x128_128x128, SCALE_BLOCK_1x128_1x128 = 0, 1, 2, 3
 SCALE_COL_MAJOR = 0
+MAJOR_K, MAJOR_MN = 0, 1
 
 _lib = None
 
@@ -58,6 +59,8 @@ def lib():
         L.fp8_scaled_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
         L.fp8_scaled_gemm_workspace_size.restype = sz
         L.fp8_scaled_gemm.argtypes = [i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, i32, p, i64, i32, p, sz, p]
+        L.fp8_scaled_gemm_ex.argtypes = [i64, i64, i64, p, i64, p, i64, i32, p, i64, p, i64, i32, i32, p, i64, i32,
+                                         p, sz, p]
         L.fp8_scaled_gemm_quant.argtypes = [i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, i32, p, i64,
                                             p, i64, p, i64, p]
         L.fp8bs_status_string.argtypes = [i32]
@@ -65,7 +68,7 @@ def lib():
         L.fp8bs_check_device_error.argtypes = [p]
         L.fp8_quant_tensor_noalloc.argtypes = [p, i32, i64, p, p, p]
         for fn in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_tensor",
-                   "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_quant",
+                   "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_ex", "fp8_scaled_gemm_quant",
                    "fp8bs_check_device_error", "fp8_quant_tensor_noalloc"):
             getattr(L, fn).restype = i32
         _lib = L
@@ -242,6 +245,41 @@ def fp8_scaled_gemm(A: torch.Tensor, Bt: torch.Tensor, scale_a: torch.Tensor, sc
                                                     scale_a.data_ptr(), ld_sa, scale_b.data_ptr(), ld_sb, mode,
                                                     SCALE_COL_MAJOR, out.data_ptr(), _ld(out), oc, wp, wn,
                                                     _stream(A)))
+    return out
+
+
+def fp8_scaled_gemm_ex(A: torch.Tensor, B: torch.Tensor, b_major: int, scale_a: torch.Tensor,
+                       scale_b: torch.Tensor, mode: int, out_dtype: torch.dtype = torch.bfloat16,
+                       out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       split_k: bool = True) -> torch.Tensor:
+    """D = scaled(A . B).  A: M x K uint8 (e4m3).  b_major = MAJOR_MN: B is the
+    K x N uint8 matrix itself (N contiguous), with a TENSOR / ROWWISE scale or
+    the ceil(K/128) x ceil(N/128) grid fp8_quant_128x128 writes for it;
+    b_major = MAJOR_K: B is B^T (N x K), exactly fp8_scaled_gemm."""
+    if b_major == MAJOR_K:
+        return fp8_scaled_gemm(A, B, scale_a, scale_b, mode, out_dtype=out_dtype, out=out, workspace=workspace,
+                               split_k=split_k)
+    M, K = A.shape
+    K2, N = B.shape
+    if K2 != K:
+        raise ValueError("A (M x K) and B (K x N) must share K")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    oc = F32 if out.dtype == torch.float32 else BF16
+    if mode in (SCALE_BLOCK_1x128_128x128, SCALE_BLOCK_1x128_1x128):
+        ld_sa = _grid_ld(scale_a, M)
+        ld_sb = _grid_ld(scale_b, scale_b.shape[0])
+    else:
+        ld_sa = ld_sb = 0
+    wsb = fp8_scaled_gemm_workspace_size(M, N, K, mode) if split_k else 0
+    if wsb > 0 and workspace is None:
+        workspace = torch.empty((wsb,), dtype=torch.uint8, device=A.device)
+    wp = workspace.data_ptr() if (workspace is not None and wsb > 0) else 0
+    wn = workspace.numel() * workspace.element_size() if (workspace is not None and wsb > 0) else 0
+    _check("fp8_scaled_gemm_ex", lib().fp8_scaled_gemm_ex(M, N, K, A.data_ptr(), _ld(A), B.data_ptr(), _ld(B),
+                                                          b_major, scale_a.data_ptr(), ld_sa, scale_b.data_ptr(),
+                                                          ld_sb, mode, SCALE_COL_MAJOR, out.data_ptr(), _ld(out),
+                                                          oc, wp, wn, _stream(A)))
     return out
 
 

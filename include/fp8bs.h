@@ -239,7 +239,7 @@ fp8bs_status fp8_quant_rowwise(const void* x, fp8bs_dtype xt, int64_t rows, int6
  * D          M x N, dtype out_dtype (bf16 rounded to nearest even, or fp32),
  *            leading dim ldd elements.
  * workspace  optional fp32 scratch for split-K (used when the output has too few
- *            128x256 tiles to fill the GPU).  Pass NULL/0 to disable split-K, or
+ *            256x128 tiles to keep the GPU's CTA pairs busy).  Pass NULL/0 to disable split-K, or
  *            at least fp8_scaled_gemm_workspace_size(M, N, K, mode) bytes.  The
  *            split partial sums are added in a fixed order: results are
  *            deterministic.
@@ -258,6 +258,43 @@ fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K,
                              fp8bs_scale_mode mode, fp8bs_scale_layout layout,
                              void* D, int64_t ldd, fp8bs_dtype out_dtype,
                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Storage order of the B operand of fp8_scaled_gemm_ex. */
+typedef enum {
+    FP8BS_MAJOR_K = 0,    /* B^T stored N x K row-major (K contiguous), as fp8_scaled_gemm takes it */
+    FP8BS_MAJOR_MN = 1    /* B stored K x N row-major (N contiguous)                               */
+} fp8bs_major;
+
+/*
+ * fp8_scaled_gemm_ex -- fp8_scaled_gemm with the storage order of B chosen by
+ * the caller: B^T (N x K, K-major, b_major = FP8BS_MAJOR_K, exactly
+ * fp8_scaled_gemm) or B itself (K x N, MN-major, b_major = FP8BS_MAJOR_MN).
+ *
+ * Defined by: the same dequantized matmul as fp8_scaled_gemm.  The MN-major
+ * form lets the backward GEMMs of the blockwise linear read an operand in the
+ * orientation it is stored in, as the blockwise linear of pytorch/ao PR #2785
+ * "integrate torch._scaled_mm into Float8BlockwiseLinear and add bench
+ * script" (Summary) consumes W and grad_out: dgrad dX = dY . W reads the
+ * forward's W_q (N_w x K_w) as B = W_q, K = N_w, N = K_w, with the forward's
+ * 128x128 scale grid, so no transposed copy of W_q is needed.
+ *
+ * With b_major = FP8BS_MAJOR_MN:
+ * B          K x N e4m3, leading dim ldb >= N (bytes), ldb % 16 == 0.
+ * scale_b    TENSOR: 1 float.  ROWWISE: N floats.
+ *            BLOCK_1x128_128x128: the grid of B's 128x128 tiles in B's storage
+ *            order, ceil(K/128) x ceil(N/128): rB(n, kb) = scale_b[kb + (n/128)*ld_sb],
+ *            ld_sb >= ceil(K/128) (as fp8_quant_128x128 writes it for the K x N
+ *            matrix).
+ *            BLOCK_1x128_1x128: FP8BS_ERR_UNSUPPORTED.
+ * Everything else (A, scale_a, D, workspace, alignment, errors) as
+ * fp8_scaled_gemm.  Asynchronous on `stream`.
+ */
+fp8bs_status fp8_scaled_gemm_ex(int64_t M, int64_t N, int64_t K,
+                                const uint8_t* A, int64_t lda, const uint8_t* B, int64_t ldb, fp8bs_major b_major,
+                                const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
+                                fp8bs_scale_mode mode, fp8bs_scale_layout layout,
+                                void* D, int64_t ldd, fp8bs_dtype out_dtype,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * fp8_scaled_gemm_quant -- the scaled GEMM with its bf16 output quantized

@@ -6,7 +6,8 @@ Cases (seeded inputs of the workloads, operands prepared before the loop so
 only the named kernel runs R times):
   gemm_fwd     Llama4 forward GEMM 16640 x 5120 x 8192, 1x128 x 128x128, bf16 out
   gemm_wgrad   Llama4 wgrad GEMM 5120 x 8192 x 16640, 1x128 x 1x128, bf16 out
-  gemm_dgrad   Llama4 dgrad GEMM 16640 x 8192 x 5120 (dy . W), 1x128 x 128x128, bf16 out
+  gemm_dgrad   Llama4 dgrad GEMM 16640 x 8192 x 5120 (dy . W), 1x128 x 128x128, bf16 out, W_q read MN-major
+  gemm_dgrad_wt        the same reading the 128x128 kernel's transposed copy of W_q (K-major)
   gemm_tensor  16640 x 5120 x 8192 per-tensor scales, bf16 out
   gemm_rowwise 16640 x 5120 x 8192 rowwise scales, bf16 out
   gemm_fwd_quant       the forward GEMM with its output quantized 1x128 in the epilogue (bf16 out stored)
@@ -74,13 +75,18 @@ def _gemm_case(name):
             mode = ops.SCALE_TENSOR
         out = torch.empty((M, 5120), dtype=torch.bfloat16, device="cuda")
         flops = 2.0 * M * 5120 * 8192
-    elif name == "gemm_dgrad":
+    elif name in ("gemm_dgrad", "gemm_dgrad_wt"):
         _, W, dy = inputs.llama4(5120, 8192)
         qa, sa = ops.fp8_quant_1x128(dy.cuda())
-        _, _, qb, sb = ops.fp8_quant_128x128(W.cuda(), want_q=False, want_qt=True)
         mode = ops.SCALE_BLOCK_1x128_128x128
         out = torch.empty((M, 8192), dtype=torch.bfloat16, device="cuda")
         flops = 2.0 * M * 8192 * 5120
+        if name == "gemm_dgrad":
+            # W_q read in its stored orientation (MN-major B)
+            qw, sw, _, _ = ops.fp8_quant_128x128(W.cuda())
+            torch.cuda.synchronize()
+            return (lambda: ops.fp8_scaled_gemm_ex(qa, qw, ops.MAJOR_MN, sa, sw, mode, out=out)), flops, "TFLOP/s"
+        _, _, qb, sb = ops.fp8_quant_128x128(W.cuda(), want_q=False, want_qt=True)
     elif name == "gemm_wgrad":
         x, _, dy = inputs.llama4(5120, 8192)
         qa, sa = ops.fp8_quant_1x128(dy.cuda(), transpose_out=True)
@@ -162,7 +168,7 @@ def _quant_case(name):
     return fn, nbytes, "GB/s"
 
 
-CONFIG_CASES = (["gemm_tiny", "gemm_pertensor_small", "gemm_rowwise_small", "gemm_fwd", "gemm_dgrad",
+CONFIG_CASES = (["gemm_tiny", "gemm_pertensor_small", "gemm_rowwise_small", "gemm_fwd", "gemm_dgrad", "gemm_dgrad_wt",
                  "gemm_wgrad", "gemm_tensor", "gemm_rowwise", "gemm_longk", "gemm_fwd_then_quant",
                  "gemm_fwd_quant", "gemm_fwd_quant_only", "quant_dual"]
                 + [f"quant_rows_{n}" for n in inputs.QUANT_SWEEP_SIZES]

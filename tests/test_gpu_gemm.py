@@ -238,14 +238,16 @@ def test_long_k_workload(K, recipe):
     assert oracle.sqnr(fp32, got.float().cpu().numpy()) >= 28.0
 
 
+@pytest.mark.parametrize("wt_copy", [True, False])
 @pytest.mark.parametrize("N,K", inputs.LLAMA4_SHAPES)
-def test_llama4_fwd_bwd_workload(N, K):
+def test_llama4_fwd_bwd_workload(N, K, wt_copy):
     """The Llama4-shape linear fwd + bwd (M = 16640) at full size, in the
-    launch configuration the benchmark times; sampled output rows of all three
-    GEMMs and sampled quantized rows against the oracle."""
+    launch configuration the benchmark times (wt_copy=True) and with dgrad
+    reading W_q MN-major instead of its transposed copy; sampled output rows
+    of all three GEMMs and sampled quantized rows against the oracle."""
     M = inputs.LLAMA4_M
     x, W, dy = inputs.llama4(N, K)
-    step = Fp8LinearStep(M, N, K)
+    step = Fp8LinearStep(M, N, K, dgrad_wt_copy=wt_copy)
     xd, Wd, dyd = x.cuda(), W.cuda(), dy.cuda()
     y, dx, dW = step.run(xd, Wd, dyd)
     torch.cuda.synchronize()
@@ -261,10 +263,14 @@ def test_llama4_fwd_bwd_workload(N, K):
     assert_bytes_equal(step.xq[torch.as_tensor(rows_m, device="cuda")], qxo, "x_q rows")
     ref = oracle.gemm(qxo, qwo, sxo, swo, oracle.SCALE_BLOCK_1x128_128x128)
     assert_bf16_close(y[torch.as_tensor(rows_m, device="cuda")], ref, "fwd")
-    # dgrad: dx = dy W  (B^T = W^T, same 128x128 tiles)
+    # dgrad: dx = dy W  (B^T = W^T, the same 128x128 tiles; without the copy
+    # the GPU reads W_q in its stored orientation)
     qdyo, sdyo = oracle.quant_1x128(dyb, rows=rows_m)
     qwto, swto = oracle.quant_128x128(Wb, transpose=True)
-    assert_bytes_equal(step.wtq, qwto, "W^T_q")
+    if wt_copy:
+        assert_bytes_equal(step.wtq, qwto, "W^T_q")
+    else:
+        assert step.wtq is None, "dgrad reads W_q without a transposed copy"
     ref = oracle.gemm(qdyo, qwto, sdyo, swto, oracle.SCALE_BLOCK_1x128_128x128)
     assert_bf16_close(dx[torch.as_tensor(rows_m, device="cuda")], ref, "dgrad")
     # wgrad: dW = dy^T x  (both quantized along tokens)
@@ -383,3 +389,75 @@ def test_gemm_quant_output(M, N, K, mode):
         torch.cuda.synchronize()
         assert torch.equal(q, q3)
         assert_scales_equal(grid_np(s), grid_np(s3), "vs fp8_quant_1x128(D)")
+
+
+# ------------------------------------------------------------------ B given MN-major (stored K x N)
+def run_random_mn(M, N, K, mode, out_dtype, seed, rows=None):
+    """D = A . B with B stored K x N (row pitch rounded up to 16 bytes) through
+    fp8_scaled_gemm_ex(MAJOR_MN); the oracle gets B^T and the scale grid in
+    its (n-block, k-block) order.  The GPU's 128x128 grid for B is the one of
+    B's storage order, (k-block, n-block)."""
+    rng = np.random.default_rng(seed)
+    A = inputs.random_e4m3_bytes(M, K, seed=seed)
+    B = inputs.random_e4m3_bytes(K, N, seed=seed + 1)
+    sa, sb = make_scales(rng, mode, M, N, K)
+    ldb = (N + 15) // 16 * 16
+    Bbuf = torch.zeros((K, ldb), dtype=torch.uint8, device="cuda")
+    Bbuf[:, :N] = B.cuda()
+    Bd = Bbuf[:, :N]
+    if mode == ops.SCALE_BLOCK_1x128_128x128:
+        sbd = to_gpu_scales(np.ascontiguousarray(sb.T), mode)      # (Kb, Nb) grid
+    else:
+        sbd = to_gpu_scales(sb, mode)
+    D = ops.fp8_scaled_gemm_ex(A.cuda(), Bd, ops.MAJOR_MN, to_gpu_scales(sa, mode), sbd, mode, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    no_device_error()
+    ref = oracle.gemm(A.numpy(), np.ascontiguousarray(B.numpy().T), sa, sb, mode, rows=rows)
+    got = D if rows is None else D[torch.as_tensor(rows, device="cuda")]
+    if out_dtype == torch.float32:
+        assert_f32_close(got, ref, f"MN-major B: M{M} N{N} K{K} mode{mode}")
+    else:
+        assert_bf16_close(got, ref, f"MN-major B: M{M} N{N} K{K} mode{mode}")
+
+
+MN_MODES = [ops.SCALE_TENSOR, ops.SCALE_ROWWISE, ops.SCALE_BLOCK_1x128_128x128]
+
+
+@pytest.mark.parametrize("mode", MN_MODES)
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (1, 1, 16), (16, 32, 32), (127, 129, 256), (129, 255, 384),
+                                   (300, 260, 1008), (64, 1000, 160), (513, 384, 2048)])
+def test_gemm_b_mn_major_shapes(M, N, K, mode):
+    """Ragged M, N and K (last K-block partial), several tiles, every recipe
+    the MN-major form supports."""
+    run_random_mn(M, N, K, mode, torch.float32, seed=3 * M + N + K + mode)
+    run_random_mn(M, N, K, mode, torch.bfloat16, seed=5 * M + N + K + mode)
+
+
+@pytest.mark.parametrize("kb", [1, 3, 64, 1001])
+def test_gemm_b_mn_major_k_blocks(kb):
+    """K-block counts up to the long-K case (split-K path at 1001)."""
+    rows = [0, 1, 77, 128, 200, 255] if kb > 64 else None
+    run_random_mn(256, 512, 128 * kb, ops.SCALE_BLOCK_1x128_128x128, torch.float32, seed=kb, rows=rows)
+
+
+def test_gemm_b_mn_major_unsupported_recipe():
+    A = torch.zeros((128, 256), dtype=torch.uint8, device="cuda")
+    B = torch.zeros((256, 128), dtype=torch.uint8, device="cuda")
+    s = ops.colmajor_grid(128, 2, "cuda").fill_(1.0)
+    with pytest.raises(ops.Fp8bsError):
+        ops.fp8_scaled_gemm_ex(A, B, ops.MAJOR_MN, s, s, ops.SCALE_BLOCK_1x128_1x128)
+
+
+def test_dgrad_mn_major_equals_transposed_copy():
+    """Llama4 dgrad (16640 x 8192 x 5120): reading W_q MN-major gives exactly
+    the output of reading the 128x128 kernel's transposed copy K-major."""
+    M = inputs.LLAMA4_M
+    _, W, dy = inputs.llama4(5120, 8192)
+    qdy, sdy = ops.fp8_quant_1x128(dy.cuda())
+    qw, sw, qwt, swt = ops.fp8_quant_128x128(W.cuda(), want_q=True, want_qt=True)
+    D_mn = ops.fp8_scaled_gemm_ex(qdy, qw, ops.MAJOR_MN, sdy, sw, ops.SCALE_BLOCK_1x128_128x128)
+    D_k = ops.fp8_scaled_gemm(qdy, qwt, sdy, swt, ops.SCALE_BLOCK_1x128_128x128)
+    torch.cuda.synchronize()
+    no_device_error()
+    assert D_mn.shape == (M, 8192)
+    assert torch.equal(D_mn, D_k)
