@@ -700,8 +700,24 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
         const int64_t chunks = M * ((N + 3) / 4);
         const int grid = (int)std::max<int64_t>(
             1, std::min<int64_t>(cdiv(chunks, kReduceThreads), (int64_t)d->num_sms * 16));
-        splitk_reduce_kernel<<<grid, kReduceThreads, 0, stream>>>(p.ws, plan.splits, M, N, plan.ldw, D, ldd,
-                                                                  p.out_f32, vec_out);
+        // programmatic dependent launch: the reduction's CTAs are scheduled
+        // while the GEMM finishes and wait in-kernel for its completion
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid, 1, 1);
+        cfg.blockDim = dim3(kReduceThreads, 1, 1);
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const float* wsp = p.ws;
+        const int splits = plan.splits;
+        const int64_t ldw = plan.ldw;
+        const int out_f32 = p.out_f32;
+        if (cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, wsp, splits, M, N, ldw, D, ldd, out_f32, vec_out) !=
+            cudaSuccess)
+            return FP8BS_ERR_CUDA;
         st = launch_status();
     }
     return st;

@@ -41,8 +41,9 @@
 //               steps: four 256x128x32 MMAs per K-block into one of the four
 //               accumulators, commits (multicast to both CTAs) each
 //               accumulator and then the smem stage.
-//   warps 4-19  promotion / epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
-//               (its rows) and 32 of the 128 columns; per accumulation group
+//   warps 4-11  promotion / epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+//               (its rows) and 64 of the 128 columns (measured faster than 16
+//               warps of 32 columns); per accumulation group
 //               (a K-block for the block recipes, one issuer's share of the K
 //               range for the tensor / rowwise recipes) it loads the partial
 //               sums, multiplies by the scale product and adds into fp32
@@ -78,13 +79,13 @@ constexpr uint32_t kPairBStage = kStepKb * kPairBTile;
 constexpr uint32_t kPairStageTx = 2 * (kPairAStage + kPairBStage);   // both CTAs' bytes per stage
 constexpr uint32_t kPairScaleKb = (kCtaM + kPairN) * 4;             // sa[128] then sb[128], per K-block
 constexpr uint32_t kPairScaleEntry = kStepKb * kPairScaleKb;
-constexpr int kPairEpiWarps = 16;
+constexpr int kPairEpiWarps = 8;
 constexpr int kPairCtrlWarps = 4;
 constexpr int kPairThreads = 32 * (kPairCtrlWarps + kPairEpiWarps);
-constexpr int kPairCols = kPairN * 4 / kPairEpiWarps;     // accumulator columns per thread (32)
+constexpr int kPairCols = kPairN * 4 / kPairEpiWarps;     // accumulator columns per thread (64)
 constexpr uint64_t kPairAbortGraceNs = 100000ull;          // abort path: time for stray loads to land
 
-static_assert(kPairCols % 32 == 0, "two 16-column TMEM loads per wait");
+static_assert(kPairCols % 32 == 0, "pairs of 16-column TMEM loads per wait");
 static_assert(kPairStages % 2 == 0 && kPairScaleStages % 2 == 0 && kPairBufs == 4,
               "stages, scale entries and accumulator pairs alternate with the step parity");
 
@@ -177,6 +178,9 @@ gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // a split-K reduction launched after this kernel may start its (waiting)
+    // CTAs now: it reads nothing before this grid has completed
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // A wait that gives up stops this CTA's roles and the peer's.
     auto give_up = [&]() {

@@ -6,8 +6,13 @@
 //
 // Memory-bound (the partials were just written by the GEMM and are normally
 // still in L2): each thread owns one 4-column chunk of a row and issues the
-// loads of eight splits before adding them in split order, so that eight
-// 16-byte loads per thread are in flight instead of one.
+// loads of up to sixteen splits before adding them in split order, so that
+// sixteen 16-byte loads per thread are in flight instead of one.
+//
+// Launched as a programmatic dependent of the GEMM (its CTAs may start while
+// the GEMM's last tiles run): griddepcontrol.wait holds every thread until the
+// GEMM grid has completed and its partial sums are visible (without that
+// launch attribute the wait returns at once).
 #pragma once
 
 #include <cstdint>
@@ -17,13 +22,14 @@
 namespace fp8bs {
 
 constexpr int kReduceThreads = 128;
-constexpr int kReduceBatch = 8;          // split loads in flight per thread
+constexpr int kReduceBatch = 16;         // split loads in flight per thread
 
 __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const float* __restrict__ ws, int splits,
                                                                        int64_t M, int64_t N, int64_t ldw,
                                                                        void* __restrict__ D, int64_t ldd, int out_f32,
                                                                        int vec_out)
 {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t nq = (N + 3) >> 2;          // 4-column chunks per row
     const int64_t total = M * nq;
     const int64_t plane = M * ldw;

@@ -14,6 +14,7 @@ only the named kernel runs R times):
   gemm_fwd_quant_only  the same without storing the bf16 output
   gemm_fwd_then_quant  the forward GEMM, then fp8_quant_1x128 of its output (two launches)
   gemm_longk   256 x 512 x 128128 (k_blocks 1001), 1x128 x 128x128, split-K, bf16 out
+  gemm_longk_mn        the same with x (K x 512) quantized as stored and read MN-major
   quant_rows   1x128 quantization of a 32768 x 32768 bf16 matrix
   quant_cols   1x128 along rows (transposed output) of a 16640 x 8192 bf16 matrix
   quant_dual   both 1x128 directions from one read of a 16640 x 8192 bf16 matrix
@@ -94,6 +95,19 @@ def _gemm_case(name):
         mode = ops.SCALE_BLOCK_1x128_1x128
         out = torch.empty((5120, 8192), dtype=torch.bfloat16, device="cuda")
         flops = 2.0 * M * 5120 * 8192
+    elif name == "gemm_longk_mn":
+        # x (K x 512) quantized 128x128 as stored and read MN-major
+        goT, x = inputs.long_k(128128)
+        qa, sa = ops.fp8_quant_1x128(goT.cuda())
+        qb, sb, _, _ = ops.fp8_quant_128x128(x.cuda())
+        mode = ops.SCALE_BLOCK_1x128_128x128
+        out = torch.empty((256, 512), dtype=torch.bfloat16, device="cuda")
+        flops = 2.0 * 256 * 512 * 128128
+        ws = ops.fp8_scaled_gemm_workspace_size(256, 512, 128128, mode)
+        wsb = torch.empty((max(ws, 16),), dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+        return (lambda: ops.fp8_scaled_gemm_ex(qa, qb, ops.MAJOR_MN, sa, sb, mode, out=out, workspace=wsb)), flops, \
+            "TFLOP/s"
     else:
         goT, x = inputs.long_k(128128)
         qa, sa = ops.fp8_quant_1x128(goT.cuda())
