@@ -38,11 +38,12 @@ UNIT = "TFLOP/s"
 PAGES_FP8_US = (7746.98, 7783.31)
 FP8_SPEC_TFLOPS = 4500.0
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
-# GEMM launch of the (5120, 8192) layer (16640 x 5120 x 8192), from an ncu
-# capture, keyed by a hash of the kernel source it was taken on.  A changed
-# kernel reports null until it is captured again.
-GEMM_TRAFFIC = {"1e8ca1a0fe545570": 572.1e6}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of each
+# GEMM of the step, from an ncu capture, keyed by a hash of the GEMM kernel
+# sources it was taken on.  A changed kernel reports null until it is captured
+# again; an old figure is never re-keyed to new sources.
+GEMM_TRAFFIC = {}
+GEMM_SOURCES = ("gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx.cuh", "splitk_reduce.cuh")
 
 
 def max_over_ranks(values, world, device):
@@ -65,7 +66,7 @@ def throughput_tflops(world, flops_per_step_per_rank, steps, ms_max):
 
 def kernel_hash():
     h = hashlib.sha256()
-    for f in ("gemm_kernel.cuh", "ptx.cuh"):
+    for f in GEMM_SOURCES:
         with open(os.path.join(ROOT, "fp8_block_scaled_11_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -225,9 +226,12 @@ def run_gpu(args):
     ms_total = t0.elapsed_time(t1)
     quant_ms = sum(e[0].elapsed_time(e[1]) for _, e in events)
     gemm_ms = sum(e[1].elapsed_time(e[4]) for _, e in events)
-    # the roofline launch: forward GEMM of the first layer shape
-    fwd_ms = sum(e[1].elapsed_time(e[2]) for st, e in events if st is steps[0])
-    ms_total, quant_ms, gemm_ms, fwd_ms = max_over_ranks([ms_total, quant_ms, gemm_ms, fwd_ms], world, "cuda")
+    # per GEMM of the step (layer shape i, GEMM g = fwd / dgrad / wgrad): summed event time
+    per_gemm_ms = [sum(e[1 + g].elapsed_time(e[2 + g]) for st, e in events if st is steps[i])
+                   for i in range(len(steps)) for g in range(3)]
+    vals = max_over_ranks([ms_total, quant_ms, gemm_ms] + per_gemm_ms, world, "cuda")
+    ms_total, quant_ms, gemm_ms, per_gemm_ms = vals[0], vals[1], vals[2], vals[3:]
+    fwd_ms = per_gemm_ms[0]
 
     flops_step = sum(st.flops() for st in steps)
     qbytes_step = sum(st.quant_bytes() for st in steps)
@@ -243,7 +247,15 @@ def run_gpu(args):
     sustained = timed_region_s > 2.0
     bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     fp8_peak = 2.0 * bf16          # fp8 / bf16 dense ratio 4.5 / 2.25
-    tr = GEMM_TRAFFIC.get(kernel_hash())
+    traffic = GEMM_TRAFFIC.get(kernel_hash(), {})
+    gemm_list = gemm_roofline_list(steps, per_gemm_ms, args.steps, fp8_peak, traffic)
+    tr = gemm_list[0]["traffic"]
+
+    # ---- sustained: the same step back to back for several seconds (the GPU
+    # settles under its power cap), against the sustained peak
+    sus = None
+    if args.sustained_s > 0:
+        sus = run_sustained(args, world, local, one_step, steps, flops_step, peaks, barrier)
 
     # ---- end to end: host (pinned) inputs -> device, the step, results -> host
     e2e = None
@@ -285,6 +297,8 @@ def run_gpu(args):
                            f"({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'fallback'}), fp8/bf16 ratio 2",
             "avg_launch_us": round(fwd_avg_us, 1),
         },
+        "roofline_gemms": gemm_list,
+        "sustained": sus,
         "clocks": clocks,
         "gpu_launches": Fp8LinearStep.LAUNCHES_PER_STEP * len(steps) * args.steps,
         "e2e": e2e,
@@ -295,6 +309,87 @@ def run_gpu(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+GEMM_NAMES = ("fwd", "dgrad", "wgrad")
+
+
+def gemm_shapes(st):
+    """(M, N, K) of the step's fwd, dgrad and wgrad GEMMs and their recipes."""
+    M, N, K = st.M, st.N, st.K
+    return ((M, N, K, "1x128 x 128x128"), (M, K, N, "1x128 x 128x128"), (N, K, M, "1x128 x 1x128"))
+
+
+def gemm_algorithmic_bytes(M, N, K, recipe):
+    """Operands read once (e4m3), scales read once, bf16 output written once."""
+    kb, nb = (K + 127) // 128, (N + 127) // 128
+    sb = nb * kb if recipe == "1x128 x 128x128" else N * kb
+    return M * K + N * K + 4 * (M * kb + sb) + 2 * M * N
+
+
+def gemm_roofline_list(steps, per_gemm_ms, nsteps, fp8_peak, traffic):
+    out = []
+    for i, st in enumerate(steps):
+        for g, (M, N, K, recipe) in enumerate(gemm_shapes(st)):
+            us = per_gemm_ms[3 * i + g] * 1e3 / nsteps
+            tflops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            key = f"{GEMM_NAMES[g]} {M}x{N}x{K}"
+            out.append({"gemm": key, "recipe": recipe,
+                        "kernel": "gemm_fp8_kernel<3>" if g == 2 else "gemm_fp8_kernel<2>",
+                        "bound": "tensor", "avg_launch_us": round(us, 1), "achieved": round(tflops, 1),
+                        "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(tflops / fp8_peak, 3),
+                        "algorithmic_bytes": gemm_algorithmic_bytes(M, N, K, recipe),
+                        "traffic": traffic.get(key)})
+    return out
+
+
+def run_sustained(args, world, local, one_step, steps, flops_step, peaks, barrier):
+    """The step back to back for at least args.sustained_s seconds of device
+    time (no per-GEMM events inside, one pair of events around each block of
+    steps), with its own clock record; the forward GEMM's share comes from a
+    final evented step.  Peak: 2 x the sustained bf16 figure."""
+    import torch
+    stream = torch.cuda.current_stream()
+    # steps per block sized from one timed step
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    one_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    est_ms = max(a.elapsed_time(b), 0.1)
+    block = max(1, int(200.0 / est_ms))
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    total_ms, nsteps = 0.0, 0
+    while total_ms < args.sustained_s * 1e3:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(block):
+            one_step()
+        b.record(stream)
+        b.synchronize()
+        total_ms += a.elapsed_time(b)
+        nsteps += block
+    # the last blocks' steps carry the settled clocks: time one more evented step
+    ev = []
+    one_step(ev)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier()
+    clocks = sampler.stop(wall0, wall1)
+    fwd_us = ev[0][1][1].elapsed_time(ev[0][1][2]) * 1e3
+    total_ms, fwd_us = max_over_ranks([total_ms, fwd_us], world, "cuda")
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
+    fwd_tflops = steps[0].gemm_flops() / (fwd_us * 1e-6) / 1e12
+    return {"seconds": round(total_ms * 1e-3, 2), "steps": nsteps, "ms_per_step": round(total_ms / nsteps, 4),
+            "value": round(throughput_tflops(world, flops_step, nsteps, total_ms), 2), "unit": UNIT,
+            "fwd_gemm_us": round(fwd_us, 1), "fwd_gemm_tflops": round(fwd_tflops, 1),
+            "fwd_frac_of_sustained_peak": round(fwd_tflops / fp8_peak, 3),
+            "peak": round(fp8_peak, 1), "peak_source": "2 x bf16_tflops_sustained (MEASURED_PEAKS.json)",
+            "clocks": clocks}
 
 
 def run_e2e(args, world, steps, shapes, data, flops_step, barrier):
@@ -439,6 +534,93 @@ def cpu_baseline_sample(rows: int, budget_s: float = 12.0):
             "seconds": round(secs, 2), "sample": f"{n} sampled steps; " + smp.describe()}
 
 
+def run_oracle_configs(args):
+    """The CPU oracle, as it stands, timed on every workload of the benchmark
+    set on this host's cores (input generation excluded): the tiny blockwise
+    GEMM, the per-tensor and rowwise GEMMs, the quantization sweep (both block
+    shapes, every size), the long-K GEMM at k_blocks 1001 (both recipes) in
+    full, and the Llama4 step on its bounded sample (as the cpu_baseline leg).
+    One JSON line per workload; then the tiny GEMM and the 4096^2 sweep point
+    again on one thread (a child process with OMP_NUM_THREADS=1)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from fp8_block_scaled_11_b200 import inputs
+
+    oracle.lib()
+    only = set(args.oracle_subset.split(",")) if args.oracle_subset else None
+    cores = _cores()
+
+    def bits(t):
+        t = t.contiguous()
+        return t.view(torch.uint16).numpy() if t.dtype == torch.bfloat16 else t.numpy()
+
+    def emit(workload, secs, work, unit, **extra):
+        d = {"workload": workload, "oracle_s": round(secs, 3), "cores": cores, "rate": work / secs, "unit": unit}
+        d.update(extra)
+        print(json.dumps(d), flush=True)
+
+    def timed(fn):
+        t = time.perf_counter()
+        r = fn()
+        return r, time.perf_counter() - t
+
+    if only is None or "tiny" in only:
+        A, Bt = inputs.tiny_blockwise()
+        Ab, Btb = bits(A), bits(Bt)
+
+        def tiny():
+            qa, sa = oracle.quant_1x128(Ab)
+            qb, sb = oracle.quant_128x128(Btb)
+            return oracle.gemm(qa, qb, sa, sb, oracle.SCALE_BLOCK_1x128_128x128)
+        _, secs = timed(tiny)
+        emit("tiny blockwise 256x512x1024 (quant + GEMM)", secs, 2.0 * 256 * 512 * 1024 / 1e12, "TFLOP/s")
+    if only is None or "pertensor" in only:
+        x, W = inputs.per_tensor()
+        xb, Wb = bits(x), bits(W)
+        for name, qf, mode in (("per-tensor", oracle.quant_tensor, oracle.SCALE_TENSOR),
+                               ("rowwise", oracle.quant_rowwise, oracle.SCALE_ROWWISE)):
+            def run():
+                qx, sx = qf(xb)
+                qw, sw = qf(Wb)
+                return oracle.gemm(qx, qw, sx, sw, mode)
+            _, secs = timed(run)
+            emit(f"{name} 256x4096x1024 (quant + GEMM)", secs, 2.0 * 256 * 4096 * 1024 / 1e12, "TFLOP/s")
+    sizes = inputs.QUANT_SWEEP_SIZES if only is None else [n for n in inputs.QUANT_SWEEP_SIZES
+                                                           if f"sweep{n}" in only]
+    for n in sizes:
+        xb = bits(inputs.quant_sweep(n))
+        for name, fn, sbytes in (("1x128", oracle.quant_1x128, 4 * n * ((n + 127) // 128)),
+                                 ("128x128", oracle.quant_128x128, 4 * ((n + 127) // 128) ** 2)):
+            _, secs = timed(lambda: fn(xb))
+            emit(f"quant {name} {n}x{n} bf16", secs, (3.0 * n * n + sbytes) / 1e9, "GB/s")
+        del xb
+    if only is None or "longk" in only:
+        K = 128128
+        goT, x = inputs.long_k(K)
+        gb, xb = bits(goT), bits(x)
+        for name, mode in (("1x128 x 128x128", oracle.SCALE_BLOCK_1x128_128x128),
+                           ("1x128 x 1x128", oracle.SCALE_BLOCK_1x128_1x128)):
+            def run():
+                qa, sa = oracle.quant_1x128(gb)
+                if mode == oracle.SCALE_BLOCK_1x128_128x128:
+                    qb, sb = oracle.quant_128x128(xb, transpose=True)
+                else:
+                    qb, sb = oracle.quant_1x128(xb, transpose=True)
+                return oracle.gemm(qa, qb, sa, sb, mode)
+            _, secs = timed(run)
+            emit(f"long-K 256x512x{K} {name} (quant + GEMM)", secs, 2.0 * 256 * 512 * K / 1e12, "TFLOP/s")
+    if only is None or "llama4" in only:
+        smp = OracleSample(args.cpu_rows)
+        flops, secs = smp.step()
+        emit("Llama4 fwd+bwd step, bounded sample", secs, flops / 1e12, "TFLOP/s", sample=smp.describe())
+    if only is None and os.environ.get("OMP_NUM_THREADS") != "1":
+        env = dict(os.environ, OMP_NUM_THREADS="1")
+        subprocess.run([sys.executable, os.path.abspath(__file__), "--oracle-configs",
+                        "--oracle-subset", "tiny,sweep4096"], env=env, check=True)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -476,10 +658,17 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sustained-s", type=float, default=3.0,
+                    help="seconds of back-to-back steps for the sustained-clock figure (0: skip)")
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="time the CPU oracle on every workload and print one JSON line per workload")
+    ap.add_argument("--oracle-subset", default="", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.oracle_configs:
+        run_oracle_configs(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
