@@ -36,7 +36,7 @@ struct DeviceInfo {
     bool sm100 = false;
     int num_sms = 0;
     int* err_ptr = nullptr;
-    std::atomic<bool> gemm_attr_set[8]{};    // per recipe, without / with the fused output quantization
+    std::atomic<bool> gemm_attr_set[16]{};   // per recipe: plain, fused output quantization, grouped
     std::atomic<int> quant_blocks[10]{};     // resident CTAs per SM, per quant kernel kind
     std::atomic<bool> tile_attr_set[8]{};
     std::atomic<int> tile_blocks[8]{};
@@ -213,13 +213,14 @@ int num_sms_current()
     return d->num_sms;
 }
 
-template <int MODE, bool QOUT = false>
+template <int MODE, bool QOUT = false, bool GROUPED = false>
 fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA,
-                         const CUtensorMap& tSB, const std::conditional_t<QOUT, GemmParamsQ, GemmParams>& p,
+                         const CUtensorMap& tSB,
+                         const std::conditional_t<QOUT, GemmParamsQ, std::conditional_t<GROUPED, GemmParamsG, GemmParams>>& p,
                          cudaStream_t stream)
 {
-    auto k = gemm_fp8_kernel<MODE, QOUT>;
-    constexpr int slot = MODE + (QOUT ? 4 : 0);
+    auto k = gemm_fp8_kernel<MODE, QOUT, GROUPED>;
+    constexpr int slot = MODE + (QOUT ? 4 : 0) + (GROUPED ? 8 : 0);
     if (!d->gemm_attr_set[slot].load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!d->gemm_attr_set[slot].load(std::memory_order_relaxed)) {
@@ -763,6 +764,76 @@ fp8bs_status fp8_scaled_gemm_quant(int64_t M, int64_t N, int64_t K, const uint8_
     qo.lds = ld_scale_out;
     return scaled_gemm(M, N, K, A, lda, Bt, ldb, false, scale_a, ld_sa, scale_b, ld_sb, mode, layout, D, ldd,
                        FP8BS_BF16, nullptr, 0, qo, stream);
+}
+
+fp8bs_status fp8_scaled_gemm_grouped(int64_t groups, const int64_t* group_rows, int64_t N, int64_t K,
+                                     const uint8_t* A, int64_t lda, const uint8_t* Bt, int64_t ldb,
+                                     const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
+                                     int64_t sb_group_stride, fp8bs_scale_mode mode, fp8bs_scale_layout layout,
+                                     void* D, int64_t ldd, fp8bs_dtype out_dtype, cudaStream_t stream)
+{
+    if (mode != FP8BS_SCALE_BLOCK_1x128_128x128 || layout != FP8BS_SCALE_COL_MAJOR || !valid_dtype(out_dtype))
+        return FP8BS_ERR_UNSUPPORTED;
+    if (groups < 1 || groups > kMaxGroups || group_rows == nullptr) return FP8BS_ERR_INVALID_ARG;
+    if (N < 1 || K < 16 || N > INT32_MAX || K > INT32_MAX || groups * N > INT32_MAX) return FP8BS_ERR_INVALID_ARG;
+    GemmParamsG p;
+    std::memset(&p, 0, sizeof p);
+    int64_t rows = 0, tiles = 0;
+    const int64_t tiles_n = cdiv(N, kBN);
+    for (int64_t g = 0; g < groups; ++g) {
+        if (group_rows[g] < 0) return FP8BS_ERR_INVALID_ARG;
+        p.row_start[g] = (int32_t)rows;
+        p.tile_start[g] = (int32_t)tiles;
+        rows += group_rows[g];
+        tiles += cdiv(group_rows[g], kBM) * tiles_n;
+        if (rows > INT32_MAX || tiles > INT32_MAX) return FP8BS_ERR_INVALID_ARG;
+    }
+    p.row_start[groups] = (int32_t)rows;
+    p.tile_start[groups] = (int32_t)tiles;
+    if (tiles == 0) return FP8BS_OK;             // every group empty: nothing to compute or write
+    if (A == nullptr || Bt == nullptr || scale_a == nullptr || scale_b == nullptr || D == nullptr)
+        return FP8BS_ERR_INVALID_ARG;
+    const int64_t Kb = cdiv(K, kBK), Nb = cdiv(N, 128);
+    if (lda < K || ldb < K || ldd < N || ld_sa < std::max<int64_t>(rows, 1) || ld_sb < Nb ||
+        sb_group_stride < ld_sb * Kb)
+        return FP8BS_ERR_INVALID_ARG;
+    if (K % 16 || lda % 16 || ldb % 16 || ld_sa % 4 || ld_sb % 4) return FP8BS_ERR_ALIGNMENT;
+    if (!aligned16(A) || !aligned16(Bt) || !aligned16(scale_a) || !aligned16(scale_b)) return FP8BS_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(D) % dtype_size(out_dtype)) return FP8BS_ERR_ALIGNMENT;
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+
+    CUtensorMap tA, tB, tSA, tSB;
+    std::memset(&tSA, 0, sizeof tSA);
+    std::memset(&tSB, 0, sizeof tSB);
+    if ((st = make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, rows, lda, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
+        return st;
+    if ((st = make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Bt, K, groups * N, ldb, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
+        return st;
+    p.M = (int32_t)rows;
+    p.N = (int32_t)N;
+    p.K = (int32_t)K;
+    p.Kb = (int32_t)Kb;
+    p.tiles_m = (int32_t)std::max<int64_t>(1, tiles);   // only the K range of decode_unit is used
+    p.tiles_n = (int32_t)tiles_n;
+    p.splits = 1;
+    p.group_m = 16;
+    p.num_units = tiles;
+    p.D = D;
+    p.ldd = ldd;
+    p.out_f32 = out_dtype == FP8BS_F32;
+    p.vec_out = aligned16(D) && (ldd * (int64_t)dtype_size(out_dtype)) % 16 == 0;
+    p.ws = nullptr;
+    p.ldw = 0;
+    p.sa = scale_a;
+    p.sb = scale_b;
+    p.ld_sa = ld_sa;
+    p.ld_sb = ld_sb;
+    p.err = d->err_ptr;
+    p.groups = (int32_t)groups;
+    p.sb_stride = sb_group_stride;
+    return launch_gemm<kModeBlock128, false, true>(d, tA, tB, tSA, tSB, p, stream);
 }
 
 }  // extern "C"

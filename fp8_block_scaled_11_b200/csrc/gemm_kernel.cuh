@@ -142,6 +142,20 @@ struct GemmParamsQ : GemmParams {
     int64_t lds_out;
 };
 
+// The grouped instantiation's parameters (a grouped / MoE GEMM: G independent
+// GEMMs D_g = scaled(A_g . B_g^T) in one persistent launch).  The groups' rows
+// of A, D and of A's scale grid are packed one after another (group g starts
+// at row row_start[g]); group g's B^T is rows g*N .. g*N + N - 1 of a stacked
+// G*N x K matrix, its 128x128 scale grid starts sb_stride floats after group
+// g-1's.  Tiles of group g are units tile_start[g] .. tile_start[g+1] - 1.
+constexpr int kMaxGroups = 64;
+struct GemmParamsG : GemmParams {
+    int32_t groups;
+    int32_t row_start[kMaxGroups + 1];
+    int32_t tile_start[kMaxGroups + 1];
+    int64_t sb_stride;
+};
+
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int64_t u, int& tm, int& tn, int& kb0, int& kb1,
                                             int& split)
 {
@@ -159,15 +173,45 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int64_t u, int&
     kb1 = (int)(((int64_t)p.Kb * (split + 1)) / p.splits);
 }
 
+// Group of unit u of a grouped launch, its tile within the group (the same
+// banded rasterization as decode_unit, over the group's tile rows), its first
+// row, one past its last row, and the first row of its B^T in the stack.
+__device__ __forceinline__ void decode_group_unit(const GemmParamsG& p, int64_t u, int& g, int& tm, int& tn,
+                                                  int& row0, int& row_end, int& brow0)
+{
+    int lo = 0, hi = p.groups - 1;
+    while (lo < hi) {                  // last group whose first tile is <= u
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.tile_start[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const int64_t local = u - p.tile_start[g];
+    row0 = p.row_start[g];
+    row_end = p.row_start[g + 1];
+    const int tiles_m = (row_end - row0 + kBM - 1) / kBM;
+    const int64_t band_tiles = (int64_t)p.group_m * p.tiles_n;
+    const int64_t band = local / band_tiles;
+    const int64_t in_band = local - band * band_tiles;
+    const int band_m0 = (int)(band * p.group_m);
+    const int band_h = min(p.group_m, tiles_m - band_m0);
+    tm = band_m0 + (int)(in_band % band_h);
+    tn = (int)(in_band / band_h);
+    brow0 = g * p.N;
+}
+
 // QOUT: the epilogue also quantizes the bf16 output, 1x128 along N (each
 // promotion thread holds one row's 128 consecutive columns: one whole group),
 // byte-identical to quantizing the stored bf16 output afterwards.
-template <int MODE, bool QOUT = false>
+// GROUPED: a grouped launch (GemmParamsG); 1x128 x 128x128 recipe, no split-K.
+// The tile's rows past its group's last row are multiplied with the next
+// group's rows of A (or TMA's zero fill) and never stored.
+template <int MODE, bool QOUT = false, bool GROUPED = false>
 __global__ void __launch_bounds__(EpiCfg<MODE>::threads, 1)
 gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                const std::conditional_t<QOUT, GemmParamsQ, GemmParams> p)
+                const std::conditional_t<QOUT, GemmParamsQ, std::conditional_t<GROUPED, GemmParamsG, GemmParams>> p)
 {
+    static_assert(!GROUPED || (MODE == kModeBlock128 && !QOUT), "grouped launches: 1x128 x 128x128, plain output");
     using E = EpiCfg<MODE>;
     static_assert(!QOUT || E::cols == 128, "fused output quantization needs one 1x128 group per thread");
     constexpr int kEpiWarps = E::warps;
@@ -268,7 +312,15 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 for (int64_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
                     int tm, tn, kb0, kb1, split;
                     decode_unit(p, u, tm, tn, kb0, kb1, split);
-                    const int m0 = tm * kBM, n0 = tn * kBN;
+                    int m0 = tm * kBM, n0 = tn * kBN;
+                    if constexpr (GROUPED) {
+                        int g, row0, row_end, brow0;
+                        decode_group_unit(p, u, g, tm, tn, row0, row_end, brow0);
+                        m0 = row0 + tm * kBM;
+                        n0 = brow0 + tn * kBN;
+                        kb0 = 0;
+                        kb1 = p.Kb;
+                    }
                     if (MODE == kModeRowwise) ok = issue_scales(m0, n0, 0);
                     for (int kb = kb0; kb < kb1 && ok; ++kb) {
                         if (!mbar_wait_bounded(ab_empty(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
@@ -371,8 +423,19 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             // 1x128 x 128x128: this thread's row scale and its columns' block
             // scale, for K-blocks kb0, kb0+1 (loaded now) and kb0+2.. (loaded
             // two groups ahead, from L2)
-            const int64_t m_glob = (int64_t)tm * kBM + row_in_tile;
-            const bool row_ok = m_glob < p.M;
+            int64_t m_glob = (int64_t)tm * kBM + row_in_tile;
+            int64_t m_end = p.M;                        // rows at or past this are never stored
+            const float* sb_g = p.sb;
+            if constexpr (GROUPED) {
+                int g, row0, row_end, brow0;
+                decode_group_unit(p, u, g, tm, tn, row0, row_end, brow0);
+                m_glob = row0 + (int64_t)tm * kBM + row_in_tile;
+                m_end = row_end;
+                sb_g = p.sb + (int64_t)g * p.sb_stride;
+                kb0 = 0;
+                kb1 = p.Kb;
+            }
+            const bool row_ok = m_glob < m_end;
             const int nb_glob = (tn * kBN + col0) / 128;
             const bool nb_ok = nb_glob * 128 < p.N;     // columns past N are never stored
             // raw values only: the product is formed when the group is promoted,
@@ -380,7 +443,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             auto load_scales = [&](int kb, float& a, float& b) {
                 if (MODE != kModeBlock128 || kb >= kb1 || !row_ok || !nb_ok) { a = b = 0.f; return; }
                 a = __ldg(p.sa + m_glob + (int64_t)kb * p.ld_sa);
-                b = __ldg(p.sb + nb_glob + (int64_t)kb * p.ld_sb);
+                b = __ldg(sb_g + nb_glob + (int64_t)kb * p.ld_sb);
             };
             float pa0, pb0, pa1, pb1;
             load_scales(kb0, pa0, pb0);
@@ -471,7 +534,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             if (!ok) break;
 
             // ---- store the tile: row m, this thread's kColsPerThread columns
-            const int64_t m = (int64_t)tm * kBM + row_in_tile;
+            const int64_t m = m_glob;
             const int n_base = tn * kBN + col0;
             if constexpr (QOUT) {
                 const int valid = p.N - n_base;            // columns of this group below N
@@ -530,7 +593,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 continue;
             }
-            if (m < p.M) {
+            if (m < m_end) {
                 if (p.splits > 1) {
                     float* dst = p.ws + ((int64_t)split * p.M + m) * p.ldw;
 #pragma unroll

@@ -61,6 +61,8 @@ def lib():
         L.fp8_scaled_gemm.argtypes = [i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, i32, p, i64, i32, p, sz, p]
         L.fp8_scaled_gemm_ex.argtypes = [i64, i64, i64, p, i64, p, i64, i32, p, i64, p, i64, i32, i32, p, i64, i32,
                                          p, sz, p]
+        L.fp8_scaled_gemm_grouped.argtypes = [i64, p, i64, i64, p, i64, p, i64, p, i64, p, i64, i64, i32, i32, p,
+                                              i64, i32, p]
         L.fp8_scaled_gemm_quant.argtypes = [i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, i32, p, i64,
                                             p, i64, p, i64, p]
         L.fp8bs_status_string.argtypes = [i32]
@@ -68,7 +70,7 @@ def lib():
         L.fp8bs_check_device_error.argtypes = [p]
         L.fp8_quant_tensor_noalloc.argtypes = [p, i32, i64, p, p, p]
         for fn in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_tensor",
-                   "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_ex", "fp8_scaled_gemm_quant",
+                   "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_ex", "fp8_scaled_gemm_quant", "fp8_scaled_gemm_grouped",
                    "fp8bs_check_device_error", "fp8_quant_tensor_noalloc"):
             getattr(L, fn).restype = i32
         _lib = L
@@ -280,6 +282,49 @@ def fp8_scaled_gemm_ex(A: torch.Tensor, B: torch.Tensor, b_major: int, scale_a: 
                                                           b_major, scale_a.data_ptr(), ld_sa, scale_b.data_ptr(),
                                                           ld_sb, mode, SCALE_COL_MAJOR, out.data_ptr(), _ld(out),
                                                           oc, wp, wn, _stream(A)))
+    return out
+
+
+def grouped_scale_grids(groups: int, N: int, K: int, device) -> torch.Tensor:
+    """Allocate the stacked 128x128 scale grids of a grouped GEMM's B: a
+    (groups, ceil(K/128), ld) fp32 tensor, ld = ceil(N/128) rounded up to 4.
+    grouped_grid_view(t, g, N) is group g's (ceil(N/128) x ceil(K/128))
+    column-major grid, the form fp8_quant_128x128 fills (out=...)."""
+    nb, kb = (N + 127) // 128, (K + 127) // 128
+    return torch.empty((groups, kb, _round_up(nb, 4)), dtype=torch.float32, device=device)
+
+
+def grouped_grid_view(t: torch.Tensor, g: int, N: int) -> torch.Tensor:
+    """Group g's grid of a grouped_scale_grids tensor: ceil(N/128) x ceil(K/128),
+    column-major (strides (1, ld))."""
+    return t[g][:, :(N + 127) // 128].t()
+
+
+def fp8_scaled_gemm_grouped(A: torch.Tensor, Bt: torch.Tensor, group_rows, scale_a: torch.Tensor,
+                            scale_b: torch.Tensor, N: int, out_dtype: torch.dtype = torch.bfloat16,
+                            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Grouped 1x128 x 128x128 GEMM: for each group g, rows of A from
+    sum(group_rows[:g]) on (group_rows[g] of them) times B_g^T = rows
+    g*N .. g*N+N-1 of Bt.  A: (sum rows) x K uint8; Bt: (G*N) x K uint8;
+    scale_a: the 1x128 grid over A's rows; scale_b: grouped_scale_grids(G, N, K).
+    Returns D (sum rows) x N."""
+    rows = [int(r) for r in group_rows]
+    G = len(rows)
+    Mt, K = A.shape
+    if Mt != sum(rows) or Bt.shape != (G * N, K):
+        raise ValueError("A must hold sum(group_rows) rows and Bt G*N rows of K bytes")
+    if scale_b.dim() != 3 or scale_b.dtype != torch.float32 or not scale_b.is_contiguous() or scale_b.shape[0] != G:
+        raise ValueError("scale_b must be grouped_scale_grids(G, N, K)")
+    if out is None:
+        out = torch.empty((Mt, N), dtype=out_dtype, device=A.device)
+    oc = F32 if out.dtype == torch.float32 else BF16
+    gr = (ctypes.c_int64 * G)(*rows)
+    ld_sa = _grid_ld(scale_a, max(Mt, 1))
+    _check("fp8_scaled_gemm_grouped",
+           lib().fp8_scaled_gemm_grouped(G, ctypes.cast(gr, ctypes.c_void_p), N, K, A.data_ptr(), _ld(A), Bt.data_ptr(),
+                                         _ld(Bt), scale_a.data_ptr(), ld_sa, scale_b.data_ptr(), scale_b.shape[2],
+                                         scale_b.shape[1] * scale_b.shape[2], SCALE_BLOCK_1x128_128x128,
+                                         SCALE_COL_MAJOR, out.data_ptr(), _ld(out), oc, _stream(A)))
     return out
 
 

@@ -327,6 +327,38 @@ fp8bs_status fp8_scaled_gemm_quant(int64_t M, int64_t N, int64_t K,
                                    void* D, int64_t ldd, uint8_t* q_out, int64_t ldq_out,
                                    float* scale_out, int64_t ld_scale_out, cudaStream_t stream);
 
+/*
+ * fp8_scaled_gemm_grouped -- G independent blockwise GEMMs in one launch (a
+ * grouped / mixture-of-experts GEMM): D_g = scaled(A_g . B_g^T), g = 0..G-1,
+ * each with the 1x128 x 128x128 recipe and its own B_g.
+ *
+ * Defined by: the grouped blockwise GEMM pytorch/ao PR #2785 "integrate
+ * torch._scaled_mm into Float8BlockwiseLinear and add bench script" mentions
+ * beside the blockwise linear (review thread: ScaledGroupedMMTensor); each
+ * group is exactly fp8_scaled_gemm with BLOCK_1x128_128x128.
+ *
+ * groups       G, 1 .. 64.
+ * group_rows   HOST array of G row counts M_g >= 0 (tokens per group; 0 allowed).
+ * A            the groups' rows packed: (sum M_g) x K e4m3, group g's first row
+ *              at sum_{h<g} M_h; leading dim lda.
+ * Bt           the groups' B^T stacked: (G*N) x K e4m3, group g at rows g*N ..
+ *              g*N+N-1; leading dim ldb.
+ * scale_a      1x128 grid over A's packed rows, scale_a[m + kb*ld_sa], ld_sa >= sum M_g.
+ * scale_b      G grids of ceil(N/128) x ceil(K/128), group g's at scale_b +
+ *              g*sb_group_stride, element [nb + kb*ld_sb]; sb_group_stride >=
+ *              ld_sb * ceil(K/128).
+ * D            (sum M_g) x N packed like A, dtype out_dtype, leading dim ldd.
+ * Recipe BLOCK_1x128_128x128 only (others: FP8BS_ERR_UNSUPPORTED).  No split-K.
+ * Alignment as fp8_scaled_gemm.  All groups empty: returns FP8BS_OK at once
+ * (the matrix pointers may then be NULL).
+ * Asynchronous on `stream`; group_rows is read before the call returns.
+ */
+fp8bs_status fp8_scaled_gemm_grouped(int64_t groups, const int64_t* group_rows, int64_t N, int64_t K,
+                                     const uint8_t* A, int64_t lda, const uint8_t* Bt, int64_t ldb,
+                                     const float* scale_a, int64_t ld_sa, const float* scale_b, int64_t ld_sb,
+                                     int64_t sb_group_stride, fp8bs_scale_mode mode, fp8bs_scale_layout layout,
+                                     void* D, int64_t ldd, fp8bs_dtype out_dtype, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* fp8bs_status_string(fp8bs_status s);
 

@@ -15,6 +15,8 @@ only the named kernel runs R times):
   gemm_fwd_then_quant  the forward GEMM, then fp8_quant_1x128 of its output (two launches)
   gemm_longk   256 x 512 x 128128 (k_blocks 1001), 1x128 x 128x128, split-K, bf16 out
   gemm_longk_mn        the same with x (K x 512) quantized as stored and read MN-major
+  gemm_grouped         grouped GEMM: 8 groups x 2080 tokens over (N, K) = (5120, 8192), 1x128 x 128x128
+  gemm_grouped_ragged  the same with ragged group sizes (4000, 1, 127, 129, 3000, 0, 5000, 4383)
   quant_rows   1x128 quantization of a 32768 x 32768 bf16 matrix
   quant_cols   1x128 along rows (transposed output) of a 16640 x 8192 bf16 matrix
   quant_dual   both 1x128 directions from one read of a 16640 x 8192 bf16 matrix
@@ -121,6 +123,25 @@ def _gemm_case(name):
     return (lambda: ops.fp8_scaled_gemm(qa, qb, sa, sb, mode, out=out, workspace=wsb)), flops, "TFLOP/s"
 
 
+def _grouped_case(name):
+    """8 groups over the Llama4 layer shape (N, K) = (5120, 8192), 16640 tokens:
+    equal counts (gemm_grouped) or ragged ones (gemm_grouped_ragged)."""
+    rows = [2080] * 8 if name == "gemm_grouped" else [4000, 1, 127, 129, 3000, 0, 5000, 4383]
+    N, K, G = 5120, 8192, len(rows)
+    x = inputs.random_matrix(sum(rows), K, seed=11, dtype=torch.bfloat16).cuda()
+    W = inputs.random_matrix(G * N, K, seed=12, dtype=torch.bfloat16, scale=K ** -0.5).cuda()
+    qa, sa = ops.fp8_quant_1x128(x)
+    qb = torch.empty((G * N, K), dtype=torch.uint8, device="cuda")
+    sb = ops.grouped_scale_grids(G, N, K, "cuda")
+    for g in range(G):
+        ops.fp8_quant_128x128(W[g * N:(g + 1) * N], out=(qb[g * N:(g + 1) * N], ops.grouped_grid_view(sb, g, N),
+                                                          None, None))
+    out = torch.empty((sum(rows), N), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    return (lambda: ops.fp8_scaled_gemm_grouped(qa, qb, rows, sa, sb, N, out=out)), 2.0 * sum(rows) * N * K, \
+        "TFLOP/s"
+
+
 def _fused_case(name):
     x, W, _ = inputs.llama4(5120, 8192)
     qa, sa = ops.fp8_quant_1x128(x.cuda())
@@ -184,7 +205,8 @@ def _quant_case(name):
 
 CONFIG_CASES = (["gemm_tiny", "gemm_pertensor_small", "gemm_rowwise_small", "gemm_fwd", "gemm_dgrad", "gemm_dgrad_wt",
                  "gemm_wgrad", "gemm_tensor", "gemm_rowwise", "gemm_longk", "gemm_fwd_then_quant",
-                 "gemm_fwd_quant", "gemm_fwd_quant_only", "quant_dual"]
+                 "gemm_fwd_quant", "gemm_fwd_quant_only", "gemm_longk_mn", "gemm_grouped", "gemm_grouped_ragged",
+                 "quant_dual"]
                 + [f"quant_rows_{n}" for n in inputs.QUANT_SWEEP_SIZES]
                 + [f"quant_tile_{n}" for n in inputs.QUANT_SWEEP_SIZES])
 
@@ -192,6 +214,8 @@ CONFIG_CASES = (["gemm_tiny", "gemm_pertensor_small", "gemm_rowwise_small", "gem
 def _case(name):
     if name in ("gemm_fwd_quant", "gemm_fwd_quant_only", "gemm_fwd_then_quant"):
         return _fused_case(name)
+    if name in ("gemm_grouped", "gemm_grouped_ragged"):
+        return _grouped_case(name)
     return _gemm_case(name) if name.startswith("gemm") else _quant_case(name)
 
 
