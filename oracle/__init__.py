@@ -28,6 +28,9 @@ SCALE_ROWWISE = 1
 SCALE_BLOCK_1x128_128x128 = 2
 SCALE_BLOCK_1x128_1x128 = 3
 
+SCALE_RULE_FP32 = 0
+SCALE_RULE_POW2 = 1
+
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
 
@@ -55,6 +58,7 @@ def lib():
         L.oracle_sqnr.restype = ctypes.c_double
         L.oracle_sqnr.argtypes = [_p, _p, _i64]
         L.oracle_to_bf16.argtypes = [_p, _i64, _p]
+        L.oracle_set_scale_rule.argtypes = [ctypes.c_int]
         _lib = L
     return _lib
 
@@ -99,6 +103,24 @@ def e4m3_decode(b: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------- #
 # Quantization.  x is a 2-D row-major array (float32, or bf16 bits as uint16).
 # --------------------------------------------------------------------------- #
+class scale_rule:
+    """Context manager selecting the quantization functions' scale rule:
+    SCALE_RULE_FP32 (the method's s = 448/amax, the default) or
+    SCALE_RULE_POW2 (the largest power of two not above it: the UE8M0 block
+    scales of hardware block scaling).  Not thread-safe (test infrastructure)."""
+
+    def __init__(self, rule: int):
+        self.rule = rule
+
+    def __enter__(self):
+        lib().oracle_set_scale_rule(self.rule)
+        return self
+
+    def __exit__(self, *exc):
+        lib().oracle_set_scale_rule(SCALE_RULE_FP32)
+        return False
+
+
 def quant_1x128(x: np.ndarray, transpose: bool = False, rows=None):
     """1x128 groups along the contiguous dim of x (or, with transpose=True,
     along the rows of x, producing the quantized transpose).

@@ -159,10 +159,32 @@ static float load_elem(const void* x, int xt, int64_t i, int64_t j, int64_t s0, 
     return ((const float*)x)[off];
 }
 
+/* Which scale rule the quantization functions apply (oracle_set_scale_rule):
+ * 0, the method's rule: s = 448 / amax in fp32;
+ * 1, the power-of-two rule of hardware block scaling (UE8M0 scale factors, an
+ *    8-bit exponent and no mantissa): s = the largest power of two not above
+ *    fl32(448 / amax), so that x * s is exact and never above 448.  This is
+ *    the B200 form of a variant without per-K-block promotion in software (the
+ *    tensor core applies power-of-two block scales itself), the counterpart of
+ *    the fast-accumulation flag of the scaled-mm template in pytorch/pytorch
+ *    issue #159940 (Describe the bug: USE_FAST_ACCUM). */
+static int g_scale_rule = 0;
+
+EXPORT void oracle_set_scale_rule(int rule)
+{
+    g_scale_rule = rule;
+}
+
 /* The scale rule for one group with absolute maximum amax. */
 static float scale_from_amax(float amax)
 {
-    return 448.0f / fmaxf(amax, 1e-12f);
+    float s = 448.0f / fmaxf(amax, 1e-12f);
+    if (g_scale_rule == 1) {
+        int e;
+        (void)frexpf(s, &e);           /* s = m * 2^e, m in [0.5, 1) */
+        s = ldexpf(1.0f, e - 1);
+    }
+    return s;
 }
 
 /* ------------------------------------------------------------------------- */
