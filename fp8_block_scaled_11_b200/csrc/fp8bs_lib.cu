@@ -1,9 +1,9 @@
 // fp8bs_lib.cu -- the C ABI declared in include/fp8bs.h: argument validation,
 // TMA tensor-map encoding, launch configuration, and the device error flag.
 // The kernels are in quant_kernels.cuh and gemm_kernel.cuh (one translation
-// unit, so the error flag is a plain __device__ variable).  The plain GEMM runs
-// on CTA pairs (gemm_pair_kernel.cuh); the GEMM with its output quantized in
-// the epilogue runs on single CTAs (gemm_kernel.cuh).
+// unit, so the error flag is a plain __device__ variable).  The GEMM runs on
+// single CTAs (gemm_kernel.cuh) or CTA pairs (gemm_pair_kernel.cuh), the
+// power-of-two block recipes on the block-scaled MMA kernel (gemm_bs_kernel.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -18,6 +18,7 @@
 #include "quant_kernels.cuh"
 #include "gemm_kernel.cuh"
 #include "gemm_pair_kernel.cuh"
+#include "gemm_bs_kernel.cuh"
 #include "splitk_reduce.cuh"
 
 using namespace fp8bs;
@@ -37,9 +38,9 @@ struct DeviceInfo {
     int num_sms = 0;
     int* err_ptr = nullptr;
     std::atomic<bool> gemm_attr_set[16]{};   // per recipe: plain, fused output quantization, grouped
-    std::atomic<int> quant_blocks[10]{};     // resident CTAs per SM, per quant kernel kind
-    std::atomic<bool> tile_attr_set[8]{};
-    std::atomic<int> tile_blocks[8]{};
+    std::atomic<int> quant_blocks[12]{};     // resident CTAs per SM, per quant kernel kind
+    std::atomic<bool> tile_attr_set[16]{};   // per tile kernel kind (+8: power-of-two scale rule)
+    std::atomic<int> tile_blocks[16]{};
     std::atomic<int> pair_clusters[8]{};     // co-resident CTA pairs, per pair-kernel instantiation
 };
 
@@ -282,44 +283,38 @@ fp8bs_status launch_pair(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap
     return launch_status();
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* fp8bs_status_string(fp8bs_status s)
+// Launch of the block-scaled MMA kernel (power-of-two recipes): one persistent
+// CTA per SM.
+template <int MODE>
+fp8bs_status launch_bs(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA,
+                       const CUtensorMap& tSB, const GemmParams& p, cudaStream_t stream)
 {
-    switch (s) {
-    case FP8BS_OK: return "FP8BS_OK";
-    case FP8BS_ERR_INVALID_ARG: return "FP8BS_ERR_INVALID_ARG";
-    case FP8BS_ERR_UNSUPPORTED: return "FP8BS_ERR_UNSUPPORTED";
-    case FP8BS_ERR_ALIGNMENT: return "FP8BS_ERR_ALIGNMENT";
-    case FP8BS_ERR_WORKSPACE: return "FP8BS_ERR_WORKSPACE";
-    case FP8BS_ERR_CUDA: return "FP8BS_ERR_CUDA";
-    case FP8BS_ERR_TIMEOUT: return "FP8BS_ERR_TIMEOUT";
-    case FP8BS_ERR_NO_SM100: return "FP8BS_ERR_NO_SM100";
+    auto k = gemm_fp8_bs_kernel<MODE>;
+    const int slot = 12 + (MODE == kModeBlock1x128 ? 1 : 0);
+    if (!d->gemm_attr_set[slot].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!d->gemm_attr_set[slot].load(std::memory_order_relaxed)) {
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BsSmem::alloc) !=
+                cudaSuccess)
+                return FP8BS_ERR_CUDA;
+            // the register hand-over is sized for exactly this allocation at launch
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return FP8BS_ERR_CUDA;
+            if (fa.numRegs != kBsLaunchRegs) return FP8BS_ERR_UNSUPPORTED;
+            d->gemm_attr_set[slot].store(true, std::memory_order_release);
+        }
     }
-    return "FP8BS_UNKNOWN_STATUS";
-}
-
-fp8bs_status fp8bs_check_device_error(cudaStream_t stream)
-{
-    DeviceInfo* d = nullptr;
-    fp8bs_status st = get_device(&d);
-    if (st != FP8BS_OK) return st;
-    if (cudaStreamSynchronize(stream) != cudaSuccess) return FP8BS_ERR_CUDA;
-    int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return FP8BS_ERR_CUDA;
-    if (v != 0) {
-        const int zero = 0;
-        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return FP8BS_ERR_CUDA;
-        return FP8BS_ERR_TIMEOUT;
-    }
-    return FP8BS_OK;
+    const int grid = (int)std::min<int64_t>(p.num_units, d->num_sms);
+    k<<<grid, kBsThreads, BsSmem::alloc, stream>>>(tA, tB, tSA, tSB, p);
+    return launch_status();
 }
 
 // ---------------------------------------------------------------- quantization
+// The group-quantization entry points, over the scale rule (POW2: the
+// power-of-two rule; the kernels are otherwise the same instantiations).
 
-fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
+template <bool POW2>
+fp8bs_status quant_1x128_impl(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
                              int64_t ldq, float* scale_inv, int64_t ld_scale, int transpose_out, cudaStream_t stream)
 {
     if (!valid_dtype(xt)) return FP8BS_ERR_UNSUPPORTED;
@@ -344,13 +339,13 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
             if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, ldx * 2, 128, 128,
                                CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
                 return st;
-            st = launch_tile_kernel(d, 6, quant_1x128_rowtile_kernel<__nv_bfloat16>, QTile<__nv_bfloat16>::smem, ctas,
+            st = launch_tile_kernel(d, 6 + (POW2 ? 8 : 0), quant_1x128_rowtile_kernel<__nv_bfloat16, POW2>, QTile<__nv_bfloat16>::smem, ctas,
                                     stream, map, rows, cols, q, ldq, scale_inv, ld_scale, d->err_ptr);
         } else {
             if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, x, cols, rows, ldx * 4, 128, 128,
                                CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
                 return st;
-            st = launch_tile_kernel(d, 7, quant_1x128_rowtile_kernel<float>, QTile<float>::smem, ctas, stream, map,
+            st = launch_tile_kernel(d, 7 + (POW2 ? 8 : 0), quant_1x128_rowtile_kernel<float, POW2>, QTile<float>::smem, ctas, stream, map,
                                     rows, cols, q, ldq, scale_inv, ld_scale, d->err_ptr);
         }
         if (st != FP8BS_OK) return st;
@@ -358,12 +353,12 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
         const int64_t items = cdiv(rows, 32) * cdiv(cols, 128);
         const int64_t ctas = cdiv(items, 8);
         if (xt == FP8BS_BF16) {
-            auto k = quant_1x128_rows_kernel<__nv_bfloat16>;
-            int g = persistent_grid(d, 0, k, ctas);
+            auto k = quant_1x128_rows_kernel<__nv_bfloat16, POW2>;
+            int g = persistent_grid(d, 0 + (POW2 ? 10 : 0), k, ctas);
             k<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
         } else {
-            auto k = quant_1x128_rows_kernel<float>;
-            int g = persistent_grid(d, 1, k, ctas);
+            auto k = quant_1x128_rows_kernel<float, POW2>;
+            int g = persistent_grid(d, 1 + (POW2 ? 10 : 0), k, ctas);
             k<<<g, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ldx, q, ldq, scale_inv, ld_scale);
         }
     } else {
@@ -373,13 +368,13 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
             if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, ldx * 2, 128, 128,
                                CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
                 return st;
-            st = launch_tile_kernel(d, 0, quant_1x128_cols_kernel<__nv_bfloat16>, QTile<__nv_bfloat16>::smem, ctas,
+            st = launch_tile_kernel(d, 0 + (POW2 ? 8 : 0), quant_1x128_cols_kernel<__nv_bfloat16, POW2>, QTile<__nv_bfloat16>::smem, ctas,
                                     stream, map, rows, cols, q, ldq, scale_inv, ld_scale, d->err_ptr);
         } else {
             if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, x, cols, rows, ldx * 4, 128, 128,
                                CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
                 return st;
-            st = launch_tile_kernel(d, 1, quant_1x128_cols_kernel<float>, QTile<float>::smem, ctas, stream, map, rows,
+            st = launch_tile_kernel(d, 1 + (POW2 ? 8 : 0), quant_1x128_cols_kernel<float, POW2>, QTile<float>::smem, ctas, stream, map, rows,
                                     cols, q, ldq, scale_inv, ld_scale, d->err_ptr);
         }
         if (st != FP8BS_OK) return st;
@@ -387,7 +382,8 @@ fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_
     return launch_status();
 }
 
-fp8bs_status fp8_quant_1x128_dual(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+template <bool POW2>
+fp8bs_status quant_1x128_dual_impl(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
                                   uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale, uint8_t* q_t,
                                   int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t, cudaStream_t stream)
 {
@@ -410,20 +406,21 @@ fp8bs_status fp8_quant_1x128_dual(const void* x, fp8bs_dtype xt, int64_t rows, i
         if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, ldx * 2, 128, 128,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
             return st;
-        st = launch_tile_kernel(d, 4, quant_1x128_dual_kernel<__nv_bfloat16>, QTile<__nv_bfloat16>::smem, ctas, stream,
+        st = launch_tile_kernel(d, 4 + (POW2 ? 8 : 0), quant_1x128_dual_kernel<__nv_bfloat16, POW2>, QTile<__nv_bfloat16>::smem, ctas, stream,
                                 map, rows, cols, q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t, ld_scale_t,
                                 d->err_ptr);
     } else {
         if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, x, cols, rows, ldx * 4, 128, 128,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
             return st;
-        st = launch_tile_kernel(d, 5, quant_1x128_dual_kernel<float>, QTile<float>::smem, ctas, stream, map, rows,
+        st = launch_tile_kernel(d, 5 + (POW2 ? 8 : 0), quant_1x128_dual_kernel<float, POW2>, QTile<float>::smem, ctas, stream, map, rows,
                                 cols, q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t, ld_scale_t, d->err_ptr);
     }
     return st;
 }
 
-fp8bs_status fp8_quant_128x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
+template <bool POW2>
+fp8bs_status quant_128x128_impl(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
                                int64_t ldq, float* scale_inv, int64_t ld_scale, uint8_t* q_t, int64_t ldq_t,
                                float* scale_inv_t, int64_t ld_scale_t, cudaStream_t stream)
 {
@@ -449,17 +446,123 @@ fp8bs_status fp8_quant_128x128(const void* x, fp8bs_dtype xt, int64_t rows, int6
         if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, cols, rows, ldx * 2, 128, 128,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
             return st;
-        st = launch_tile_kernel(d, 2, quant_128x128_kernel<__nv_bfloat16>, QTile<__nv_bfloat16>::smem, ctas, stream,
+        st = launch_tile_kernel(d, 2 + (POW2 ? 8 : 0), quant_128x128_kernel<__nv_bfloat16, POW2>, QTile<__nv_bfloat16>::smem, ctas, stream,
                                 map, rows, cols, q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t, ld_scale_t,
                                 d->err_ptr);
     } else {
         if ((st = make_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, x, cols, rows, ldx * 4, 128, 128,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK)
             return st;
-        st = launch_tile_kernel(d, 3, quant_128x128_kernel<float>, QTile<float>::smem, ctas, stream, map, rows, cols,
+        st = launch_tile_kernel(d, 3 + (POW2 ? 8 : 0), quant_128x128_kernel<float, POW2>, QTile<float>::smem, ctas, stream, map, rows, cols,
                                 q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t, ld_scale_t, d->err_ptr);
     }
     return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fp8bs_status_string(fp8bs_status s)
+{
+    switch (s) {
+    case FP8BS_OK: return "FP8BS_OK";
+    case FP8BS_ERR_INVALID_ARG: return "FP8BS_ERR_INVALID_ARG";
+    case FP8BS_ERR_UNSUPPORTED: return "FP8BS_ERR_UNSUPPORTED";
+    case FP8BS_ERR_ALIGNMENT: return "FP8BS_ERR_ALIGNMENT";
+    case FP8BS_ERR_WORKSPACE: return "FP8BS_ERR_WORKSPACE";
+    case FP8BS_ERR_CUDA: return "FP8BS_ERR_CUDA";
+    case FP8BS_ERR_TIMEOUT: return "FP8BS_ERR_TIMEOUT";
+    case FP8BS_ERR_NO_SM100: return "FP8BS_ERR_NO_SM100";
+    case FP8BS_ERR_SCALE: return "FP8BS_ERR_SCALE";
+    }
+    return "FP8BS_UNKNOWN_STATUS";
+}
+
+fp8bs_status fp8bs_check_device_error(cudaStream_t stream)
+{
+    DeviceInfo* d = nullptr;
+    fp8bs_status st = get_device(&d);
+    if (st != FP8BS_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return FP8BS_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return FP8BS_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return FP8BS_ERR_CUDA;
+        // bit 0: a bounded wait ran out; bit 1: a power-of-two recipe met another scale
+        return (v & 1) || !(v & 2) ? FP8BS_ERR_TIMEOUT : FP8BS_ERR_SCALE;
+    }
+    return FP8BS_OK;
+}
+
+// ---------------------------------------------------------------- quantization
+
+fp8bs_status fp8_quant_1x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
+                             int64_t ldq, float* scale_inv, int64_t ld_scale, int transpose_out, cudaStream_t stream)
+{
+    return quant_1x128_impl<false>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, transpose_out, stream);
+}
+
+fp8bs_status fp8_quant_1x128_ex(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
+                                int64_t ldq, float* scale_inv, int64_t ld_scale, int transpose_out,
+                                fp8bs_scale_rule rule, cudaStream_t stream)
+{
+    switch (rule) {
+    case FP8BS_SCALE_RULE_FP32:
+        return quant_1x128_impl<false>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, transpose_out, stream);
+    case FP8BS_SCALE_RULE_POW2:
+        return quant_1x128_impl<true>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, transpose_out, stream);
+    }
+    return FP8BS_ERR_UNSUPPORTED;
+}
+
+fp8bs_status fp8_quant_1x128_dual(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                                  uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale, uint8_t* q_t,
+                                  int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t, cudaStream_t stream)
+{
+    return quant_1x128_dual_impl<false>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, q_t, ldq_t,
+                                        scale_inv_t, ld_scale_t, stream);
+}
+
+fp8bs_status fp8_quant_1x128_dual_ex(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                                     uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale, uint8_t* q_t,
+                                     int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t, fp8bs_scale_rule rule,
+                                     cudaStream_t stream)
+{
+    switch (rule) {
+    case FP8BS_SCALE_RULE_FP32:
+        return quant_1x128_dual_impl<false>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, q_t, ldq_t,
+                                            scale_inv_t, ld_scale_t, stream);
+    case FP8BS_SCALE_RULE_POW2:
+        return quant_1x128_dual_impl<true>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, q_t, ldq_t,
+                                           scale_inv_t, ld_scale_t, stream);
+    }
+    return FP8BS_ERR_UNSUPPORTED;
+}
+
+fp8bs_status fp8_quant_128x128(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx, uint8_t* q,
+                               int64_t ldq, float* scale_inv, int64_t ld_scale, uint8_t* q_t, int64_t ldq_t,
+                               float* scale_inv_t, int64_t ld_scale_t, cudaStream_t stream)
+{
+    return quant_128x128_impl<false>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, q_t, ldq_t, scale_inv_t,
+                                     ld_scale_t, stream);
+}
+
+fp8bs_status fp8_quant_128x128_ex(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                                  uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale, uint8_t* q_t,
+                                  int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t, fp8bs_scale_rule rule,
+                                  cudaStream_t stream)
+{
+    switch (rule) {
+    case FP8BS_SCALE_RULE_FP32:
+        return quant_128x128_impl<false>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, q_t, ldq_t,
+                                         scale_inv_t, ld_scale_t, stream);
+    case FP8BS_SCALE_RULE_POW2:
+        return quant_128x128_impl<true>(x, xt, rows, cols, ldx, q, ldq, scale_inv, ld_scale, q_t, ldq_t,
+                                        scale_inv_t, ld_scale_t, stream);
+    }
+    return FP8BS_ERR_UNSUPPORTED;
 }
 
 size_t fp8_quant_tensor_workspace_size(int64_t n)
@@ -526,9 +629,11 @@ fp8bs_status fp8_quant_rowwise(const void* x, fp8bs_dtype xt, int64_t rows, int6
 
 size_t fp8_scaled_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8bs_scale_mode mode)
 {
-    (void)mode;
     if (M < 1 || N < 1 || K < 1) return 0;
     const int sms = num_sms_current();
+    // the power-of-two recipes run on single CTAs only
+    if (mode == FP8BS_SCALE_BLOCK_1x128_128x128_POW2 || mode == FP8BS_SCALE_BLOCK_1x128_1x128_POW2)
+        return plan_gemm(M, N, K, sms).ws_bytes;
     // the larger of the two kernels' needs: fp8_scaled_gemm_ex with an
     // MN-major B always runs the pair kernel
     return std::max(plan_pair(M, N, K, sms).ws_bytes,
@@ -554,7 +659,11 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
                          cudaStream_t stream)
 {
     const bool quant_out = qo.q != nullptr;
-    if (mode < FP8BS_SCALE_TENSOR || mode > FP8BS_SCALE_BLOCK_1x128_1x128) return FP8BS_ERR_UNSUPPORTED;
+    if (mode < FP8BS_SCALE_TENSOR || mode > FP8BS_SCALE_BLOCK_1x128_1x128_POW2) return FP8BS_ERR_UNSUPPORTED;
+    // the power-of-two recipes: the block recipes' scale grids, block-scaled MMA
+    const bool pow2 = mode == FP8BS_SCALE_BLOCK_1x128_128x128_POW2 || mode == FP8BS_SCALE_BLOCK_1x128_1x128_POW2;
+    if (pow2 && (quant_out || b_mn)) return FP8BS_ERR_UNSUPPORTED;
+    const bool grid128 = mode == FP8BS_SCALE_BLOCK_1x128_128x128 || mode == FP8BS_SCALE_BLOCK_1x128_128x128_POW2;
     if (layout != FP8BS_SCALE_COL_MAJOR || !valid_dtype(out_dtype)) return FP8BS_ERR_UNSUPPORTED;
     if (quant_out && (mode == FP8BS_SCALE_BLOCK_1x128_1x128 || out_dtype != FP8BS_BF16)) return FP8BS_ERR_UNSUPPORTED;
     if (b_mn && (quant_out || mode == FP8BS_SCALE_BLOCK_1x128_1x128)) return FP8BS_ERR_UNSUPPORTED;
@@ -568,11 +677,11 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
         if (!aligned16(qo.q) || !aligned16(qo.s) || qo.ldq % 16 || qo.lds % 4) return FP8BS_ERR_ALIGNMENT;
     }
     const int64_t Kb = cdiv(K, kBK), Nb = cdiv(N, 128);
-    const bool block = (mode == FP8BS_SCALE_BLOCK_1x128_128x128 || mode == FP8BS_SCALE_BLOCK_1x128_1x128);
+    const bool block = (mode == FP8BS_SCALE_BLOCK_1x128_128x128 || mode == FP8BS_SCALE_BLOCK_1x128_1x128 || pow2);
     if (block) {
         if (ld_sa < M) return FP8BS_ERR_INVALID_ARG;
-        if (mode == FP8BS_SCALE_BLOCK_1x128_128x128 && ld_sb < (b_mn ? Kb : Nb)) return FP8BS_ERR_INVALID_ARG;
-        if (mode == FP8BS_SCALE_BLOCK_1x128_1x128 && ld_sb < N) return FP8BS_ERR_INVALID_ARG;
+        if (grid128 && ld_sb < (b_mn ? Kb : Nb)) return FP8BS_ERR_INVALID_ARG;
+        if (!grid128 && ld_sb < N) return FP8BS_ERR_INVALID_ARG;
         if (ld_sa % 4 || ld_sb % 4) return FP8BS_ERR_ALIGNMENT;
     }
     if (K % 16 || lda % 16 || ldb % 16) return FP8BS_ERR_ALIGNMENT;
@@ -584,7 +693,7 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
     if (st != FP8BS_OK) return st;
 
     // single-CTA tiles (128 x 256) or CTA pairs (256 x 128)
-    const bool pair = use_pair(M, N, K, b_mn, quant_out, d->num_sms);
+    const bool pair = !pow2 && use_pair(M, N, K, b_mn, quant_out, d->num_sms);
     SplitPlan plan = pair ? plan_pair(M, N, K, d->num_sms) : plan_gemm(M, N, K, d->num_sms);
     if (quant_out) plan.splits = 1;              // the epilogue quantizes whole tiles
     if (plan.splits > 1) {
@@ -639,6 +748,17 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
         if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, sa_box, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
         if ((st = make_map(&tSB, f32, 4, scale_b, N, Kb, ld_sb * 4, sb_box, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
         break;
+    case FP8BS_SCALE_BLOCK_1x128_128x128_POW2:
+    case FP8BS_SCALE_BLOCK_1x128_1x128_POW2:
+        // block-scaled kernel: four K-blocks of each grid per load (rows x 4,
+        // or the aligned group of four 128-column blocks of B x 4)
+        if ((st = make_map(&tSA, f32, 4, scale_a, M, Kb, ld_sa * 4, kBM, kSfKb, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        if (grid128) {
+            if ((st = make_map(&tSB, f32, 4, scale_b, Nb, Kb, ld_sb * 4, 4, kSfKb, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) return st;
+        } else if ((st = make_map(&tSB, f32, 4, scale_b, N, Kb, ld_sb * 4, kBN, kSfKb, CU_TENSOR_MAP_SWIZZLE_NONE)) != FP8BS_OK) {
+            return st;
+        }
+        break;
     }
 
     GemmParamsQ p;
@@ -675,7 +795,10 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
         }
     }
     const GemmParams& pb = p;                    // the plain kernels take the base block
-    if (!pair) {
+    if (pow2) {
+        st = mode == FP8BS_SCALE_BLOCK_1x128_128x128_POW2 ? launch_bs<kModeBlock128>(d, tA, tB, tSA, tSB, pb, stream)
+                                                          : launch_bs<kModeBlock1x128>(d, tA, tB, tSA, tSB, pb, stream);
+    } else if (!pair) {
         switch (mode) {
         case FP8BS_SCALE_TENSOR: st = launch_gemm<kModeTensor>(d, tA, tB, tSA, tSB, pb, stream); break;
         case FP8BS_SCALE_ROWWISE: st = launch_gemm<kModeRowwise>(d, tA, tB, tSA, tSB, pb, stream); break;

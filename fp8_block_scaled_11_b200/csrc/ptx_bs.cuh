@@ -1,0 +1,73 @@
+// ptx_bs.cuh -- inline-PTX wrappers of the block-scaled MMA path (sm_100a):
+// the kind::mxf8f6f4.block_scale instruction and its descriptor, stores into
+// TMEM, and a register fence for 32-column TMEM loads.  Single instructions,
+// as in ptx.cuh; used by gemm_bs_kernel.cuh only.
+#pragma once
+
+#include <cstdint>
+#include "ptx.cuh"
+
+namespace fp8bs {
+
+// ------------------------------------------------------------------ block-scaled MMA
+// kind::mxf8f6f4.block_scale (one scale factor per 32 consecutive K of each
+// row of A and of B^T, UE8M0: an 8-bit biased exponent, the value 2^(e-127)).
+// The instruction descriptor of this kind has no D-format field (D is F32):
+// bits [4,6) the B scale-factor id, [7,10) / [10,13) A / B format (E4M3 = 0),
+// 15 / 16 A / B major (K = 0), [17,23) N >> 3, bit 23 the scale type
+// (1 = UE8M0), [24,29) M >> 4, [29,31) the A scale-factor id.  The id selects
+// the byte of each 32-bit TMEM scale-factor word that this MMA uses.
+__host__ __device__ constexpr uint32_t idesc_e4m3_bs(uint32_t M, uint32_t N, uint32_t sf_id)
+{
+    return (sf_id << 4)
+         | (0u << 7) | (0u << 10)
+         | (0u << 15) | (0u << 16)
+         | ((N >> 3) << 17)
+         | (1u << 23)
+         | ((M >> 4) << 24)
+         | (sf_id << 29);
+}
+
+// D[tmem] (+)= (A[smem] . B[smem]^T) with each product scaled by its rows'
+// scale factors, read from TMEM at sfa / sfb (the scale-factor byte id is
+// carried in bits [30,32) of these addresses as well as in the descriptor).
+__device__ __forceinline__ void umma_f8_bs(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t sfa, uint32_t sfb, uint32_t accum)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns: thread i of the warp writes
+// r[0..15] to columns [col, col+16) of TMEM lane (lane_base + i).
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// Waits for this thread's outstanding tcgen05.st.
+__device__ __forceinline__ void tmem_st_wait()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// reg_after_wait for the 32 destination registers of a 32-column load.
+__device__ __forceinline__ void reg_after_wait32(uint32_t (&r)[32])
+{
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                   "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
+}  // namespace fp8bs

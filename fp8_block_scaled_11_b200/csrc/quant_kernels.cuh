@@ -3,6 +3,8 @@
 // One rule for every group shape: amax = max|x| over the group, s = 448 /
 // max(amax, 1e-12) (IEEE fp32 division), q = e4m3(x * s) with round-to-
 // nearest-even and saturation (cvt.rn.satfinite), stored scale = 1/s (IEEE).
+// The group kernels also have a POW2 instantiation that rounds s down to a
+// power of two first (scale_rule), for the GEMM's power-of-two recipes.
 // Group shapes follow pytorch/ao PR #2592 "add more generic kernel for fp8
 // blockwise scaling" (Performance table: (1,128) and (128,128)); reciprocal,
 // column-major scales follow pytorch/ao PR #2785 "integrate torch._scaled_mm
@@ -26,6 +28,18 @@ constexpr float kAmaxFloor = 1e-12f;
 __device__ __forceinline__ float scale_from_amax(float amax)
 {
     return __fdiv_rn(kE4M3Max, fmaxf(amax, kAmaxFloor));
+}
+
+// The power-of-two rule (POW2): the largest power of two not above the fp32
+// scale, so that the reciprocal is exactly representable as a UE8M0 scale
+// factor (8-bit biased exponent, the scale type of the tensor cores' block-
+// scaled MMA).  s is positive and normal (amax is floored at 1e-12 and
+// finite), so clearing its mantissa bits gives that power of two.
+template <bool POW2>
+__device__ __forceinline__ float scale_rule(float amax)
+{
+    const float s = scale_from_amax(amax);
+    return POW2 ? __uint_as_float(__float_as_uint(s) & 0x7F800000u) : s;
 }
 
 // 8 consecutive inputs as fp32.  bf16: one 16-byte load; fp32: two.
@@ -93,7 +107,7 @@ __device__ __forceinline__ uint2 quant8(const float (&f)[8], float s)
 // are broadcast back by shuffles.  A batch's 16 reciprocal scales (adjacent in
 // the column-major grid) leave in one coalesced 64-byte store.
 // --------------------------------------------------------------------------
-template <typename T>
+template <typename T, bool POW2 = false>
 __global__ void __launch_bounds__(256) quant_1x128_rows_kernel(
     const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ldx,
     uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sinv, int64_t ld_s)
@@ -134,7 +148,7 @@ __global__ void __launch_bounds__(256) quant_1x128_rows_kernel(
                 const float other = __shfl_sync(0xffffffffu, amax, (lane & 1) << 4);
                 if ((lane >> 1) == i) my_amax = other;
             }
-            const float my_s = scale_from_amax(my_amax);
+            const float my_s = scale_rule<POW2>(my_amax);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int64_t r = (rb << 5) + (b << 4) + (i << 1) + half;
@@ -313,7 +327,7 @@ __device__ __forceinline__ void qblock_coords(int& strip, int& group, int& wr, i
 // output row c (input column c) is input rows [128 t, 128 t + 128).  Column
 // maxima: the thread's 8 rows, the warp's 4 row groups (shuffles), the 4
 // warps holding the tile's 32-row quarters (shared memory).
-template <typename T>
+template <typename T, bool POW2 = false>
 __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(
     const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
     uint8_t* __restrict__ qt, int64_t ldq, float* __restrict__ sinv, int64_t ld_s, int* err)
@@ -345,7 +359,7 @@ __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(
         // one scale per output row (tile column): threads 0..127
         if (threadIdx.x < 128) {
             const int c = threadIdx.x;
-            const float sc = scale_from_amax(fmaxf(fmaxf(s_part[0][c], s_part[1][c]), fmaxf(s_part[2][c], s_part[3][c])));
+            const float sc = scale_rule<POW2>(fmaxf(fmaxf(s_part[0][c], s_part[1][c]), fmaxf(s_part[2][c], s_part[3][c])));
             s_scale[c] = sc;
             const int64_t cg = (tc << 7) + c;
             if (cg < cols) sinv[cg + tr * ld_s] = __frcp_rn(sc);
@@ -370,7 +384,7 @@ __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(
 // columns, the warp's 8 strips (shuffles) and the tile's two 64-column halves
 // (shared memory).  Byte-identical to quant_1x128_rows_kernel; used when the
 // row count is a multiple of 16.
-template <typename T>
+template <typename T, bool POW2 = false>
 __global__ void __launch_bounds__(256) quant_1x128_rowtile_kernel(
     const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
     uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sinv, int64_t ld_s, int* err)
@@ -405,7 +419,7 @@ __global__ void __launch_bounds__(256) quant_1x128_rowtile_kernel(
         release();
         if (threadIdx.x < 128) {
             const int r = threadIdx.x;
-            const float sr = scale_from_amax(fmaxf(s_rpart[0][r], s_rpart[1][r]));
+            const float sr = scale_rule<POW2>(fmaxf(s_rpart[0][r], s_rpart[1][r]));
             s_rscale[r] = sr;
             const int64_t rg = (tr << 7) + r;
             if (rg < rows) sinv[rg + tc * ld_s] = __frcp_rn(sr);
@@ -432,7 +446,7 @@ __global__ void __launch_bounds__(256) quant_1x128_rowtile_kernel(
 // thread's 8 columns, the warp's 8 strips (shuffles) and the tile's two
 // 64-column halves (shared memory).  Outputs are byte-identical to the
 // row-direction and transposed column-direction launches.
-template <typename T>
+template <typename T, bool POW2 = false>
 __global__ void __launch_bounds__(256) quant_1x128_dual_kernel(
     const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
     uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sinv, int64_t ld_s,
@@ -481,13 +495,13 @@ __global__ void __launch_bounds__(256) quant_1x128_dual_kernel(
         // threads 0..127: one scale per tile column; 128..255: one per tile row
         if (threadIdx.x < 128) {
             const int c = threadIdx.x;
-            const float sc = scale_from_amax(fmaxf(fmaxf(s_cpart[0][c], s_cpart[1][c]), fmaxf(s_cpart[2][c], s_cpart[3][c])));
+            const float sc = scale_rule<POW2>(fmaxf(fmaxf(s_cpart[0][c], s_cpart[1][c]), fmaxf(s_cpart[2][c], s_cpart[3][c])));
             s_cscale[c] = sc;
             const int64_t cg = (tc << 7) + c;
             if (cg < cols) sinvt[cg + tr * ld_st] = __frcp_rn(sc);
         } else {
             const int r = threadIdx.x - 128;
-            const float sr = scale_from_amax(fmaxf(s_rpart[0][r], s_rpart[1][r]));
+            const float sr = scale_rule<POW2>(fmaxf(s_rpart[0][r], s_rpart[1][r]));
             s_rscale[r] = sr;
             const int64_t rg = (tr << 7) + r;
             if (rg < rows) sinv[rg + tc * ld_s] = __frcp_rn(sr);
@@ -515,7 +529,7 @@ __global__ void __launch_bounds__(256) quant_1x128_dual_kernel(
 
 // 128x128 tiles: amax over the tile (shuffles + shared memory), then
 // row-major and/or transposed bytes straight from registers.
-template <typename T>
+template <typename T, bool POW2 = false>
 __global__ void __launch_bounds__(256) quant_128x128_kernel(
     const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
     uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sinv, int64_t ld_s,
@@ -545,7 +559,7 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(
         float amax = s_warp[0];
 #pragma unroll
         for (int w = 1; w < 8; ++w) amax = fmaxf(amax, s_warp[w]);
-        const float s = scale_from_amax(amax);
+        const float s = scale_rule<POW2>(amax);
         const int64_t r0 = (bi << 7) + 8 * group;
         const int64_t c0 = (bj << 7) + 8 * strip;
         const bool in = c0 < cols && r0 < rows;    // rows, cols % 16 == 0: blocks are all-in or all-out

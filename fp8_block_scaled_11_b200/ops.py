@@ -24,10 +24,16 @@ FP8BS_OK = 0
 STATUS_NAMES = {
     0: "FP8BS_OK", 1: "FP8BS_ERR_INVALID_ARG", 2: "FP8BS_ERR_UNSUPPORTED", 3: "FP8BS_ERR_ALIGNMENT",
     4: "FP8BS_ERR_WORKSPACE", 5: "FP8BS_ERR_CUDA", 6: "FP8BS_ERR_TIMEOUT", 7: "FP8BS_ERR_NO_SM100",
+    8: "FP8BS_ERR_SCALE",
 }
 
 BF16, F32 = 0, 1
 SCALE_TENSOR, SCALE_ROWWISE, SCALE_BLOCK_1x128_128x128, SCALE_BLOCK_1x128_1x128 = 0, 1, 2, 3
+# the block recipes with power-of-two scales on the block-scaled MMA
+SCALE_BLOCK_1x128_128x128_POW2, SCALE_BLOCK_1x128_1x128_POW2 = 4, 5
+BLOCK_MODES = (SCALE_BLOCK_1x128_128x128, SCALE_BLOCK_1x128_1x128,
+               SCALE_BLOCK_1x128_128x128_POW2, SCALE_BLOCK_1x128_1x128_POW2)
+SCALE_RULE_FP32, SCALE_RULE_POW2 = 0, 1
 SCALE_COL_MAJOR = 0
 MAJOR_K, MAJOR_MN = 0, 1
 
@@ -52,6 +58,9 @@ def lib():
         L.fp8_quant_1x128.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, i32, p]
         L.fp8_quant_1x128_dual.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, p, i64, p, i64, p]
         L.fp8_quant_128x128.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, p, i64, p, i64, p]
+        L.fp8_quant_1x128_ex.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, i32, i32, p]
+        L.fp8_quant_1x128_dual_ex.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, p]
+        L.fp8_quant_128x128_ex.argtypes = [p, i32, i64, i64, i64, p, i64, p, i64, p, i64, p, i64, i32, p]
         L.fp8_quant_tensor_workspace_size.argtypes = [i64]
         L.fp8_quant_tensor_workspace_size.restype = sz
         L.fp8_quant_tensor.argtypes = [p, i32, i64, p, p, p, sz, p]
@@ -69,7 +78,8 @@ def lib():
         L.fp8bs_status_string.restype = ctypes.c_char_p
         L.fp8bs_check_device_error.argtypes = [p]
         L.fp8_quant_tensor_noalloc.argtypes = [p, i32, i64, p, p, p]
-        for fn in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_tensor",
+        for fn in ("fp8_quant_1x128", "fp8_quant_1x128_dual", "fp8_quant_128x128", "fp8_quant_1x128_ex",
+                   "fp8_quant_1x128_dual_ex", "fp8_quant_128x128_ex", "fp8_quant_tensor",
                    "fp8_quant_rowwise", "fp8_scaled_gemm", "fp8_scaled_gemm_ex", "fp8_scaled_gemm_quant", "fp8_scaled_gemm_grouped",
                    "fp8bs_check_device_error", "fp8_quant_tensor_noalloc"):
             getattr(L, fn).restype = i32
@@ -122,11 +132,12 @@ def _grid_ld(s: torch.Tensor, rows: int) -> int:
 
 # ---------------------------------------------------------------------------- quantization
 def fp8_quant_1x128(x: torch.Tensor, transpose_out: bool = False, q: Optional[torch.Tensor] = None,
-                    scale_inv: Optional[torch.Tensor] = None):
+                    scale_inv: Optional[torch.Tensor] = None, rule: int = SCALE_RULE_FP32):
     """Returns (q uint8, scale_inv grid).  transpose_out=False: q is rows x cols,
     grid rows x ceil(cols/128).  transpose_out=True: groups run along rows and
     q is the quantized transpose (cols x rows), grid cols x ceil(rows/128).
-    Preallocated outputs may be passed as q / scale_inv."""
+    Preallocated outputs may be passed as q / scale_inv.  rule =
+    SCALE_RULE_POW2 rounds every scale down to a power of two (fp8_quant_1x128_ex)."""
     rows, cols = x.shape
     xt = _dtype_code(x)
     out_rows, out_cols = (cols, rows) if transpose_out else (rows, cols)
@@ -134,16 +145,22 @@ def fp8_quant_1x128(x: torch.Tensor, transpose_out: bool = False, q: Optional[to
         q = torch.empty((out_rows, out_cols), dtype=torch.uint8, device=x.device)
     s = scale_inv if scale_inv is not None else colmajor_grid(out_rows, (out_cols + 127) // 128, x.device)
     ld_s = _grid_ld(s, out_rows)
-    _check("fp8_quant_1x128", lib().fp8_quant_1x128(x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(), q.stride(0),
-                                                    s.data_ptr(), ld_s, int(transpose_out), _stream(x)))
+    if rule == SCALE_RULE_FP32:
+        _check("fp8_quant_1x128", lib().fp8_quant_1x128(x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(),
+                                                        q.stride(0), s.data_ptr(), ld_s, int(transpose_out),
+                                                        _stream(x)))
+    else:
+        _check("fp8_quant_1x128_ex", lib().fp8_quant_1x128_ex(x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(),
+                                                              q.stride(0), s.data_ptr(), ld_s, int(transpose_out),
+                                                              int(rule), _stream(x)))
     return q, s
 
 
-def fp8_quant_1x128_dual(x: torch.Tensor, out=None):
+def fp8_quant_1x128_dual(x: torch.Tensor, out=None, rule: int = SCALE_RULE_FP32):
     """Both 1x128 quantizations from one read of x: returns (q, scale_inv,
     q_t, scale_inv_t), equal to fp8_quant_1x128(x) followed by
     fp8_quant_1x128(x, transpose_out=True).  Preallocated outputs may be
-    passed as out=(q, scale_inv, q_t, scale_inv_t)."""
+    passed as out=(q, scale_inv, q_t, scale_inv_t).  rule as fp8_quant_1x128."""
     rows, cols = x.shape
     xt = _dtype_code(x)
     if out is None:
@@ -153,18 +170,22 @@ def fp8_quant_1x128_dual(x: torch.Tensor, out=None):
         st = colmajor_grid(cols, (rows + 127) // 128, x.device)
     else:
         q, s, qt, st = out
-    _check("fp8_quant_1x128_dual",
-           lib().fp8_quant_1x128_dual(x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(), q.stride(0), s.data_ptr(),
-                                      _grid_ld(s, rows), qt.data_ptr(), qt.stride(0), st.data_ptr(), _grid_ld(st, cols),
-                                      _stream(x)))
+    args = (x.data_ptr(), xt, rows, cols, _ld(x), q.data_ptr(), q.stride(0), s.data_ptr(), _grid_ld(s, rows),
+            qt.data_ptr(), qt.stride(0), st.data_ptr(), _grid_ld(st, cols))
+    if rule == SCALE_RULE_FP32:
+        _check("fp8_quant_1x128_dual", lib().fp8_quant_1x128_dual(*args, _stream(x)))
+    else:
+        _check("fp8_quant_1x128_dual_ex", lib().fp8_quant_1x128_dual_ex(*args, int(rule), _stream(x)))
     return q, s, qt, st
 
 
-def fp8_quant_128x128(x: torch.Tensor, want_q: bool = True, want_qt: bool = False, out=None):
+def fp8_quant_128x128(x: torch.Tensor, want_q: bool = True, want_qt: bool = False, out=None,
+                      rule: int = SCALE_RULE_FP32):
     """Returns (q, scale_inv, q_t, scale_inv_t); the unrequested pair is None.
     q: rows x cols, grid ceil(rows/128) x ceil(cols/128).  q_t: cols x rows
     (the same quantized tiles transposed), grid ceil(cols/128) x ceil(rows/128).
-    Preallocated outputs may be passed as out=(q, s, q_t, s_t)."""
+    Preallocated outputs may be passed as out=(q, s, q_t, s_t).  rule as
+    fp8_quant_1x128."""
     rows, cols = x.shape
     xt = _dtype_code(x)
     rb, cb = (rows + 127) // 128, (cols + 127) // 128
@@ -183,8 +204,11 @@ def fp8_quant_128x128(x: torch.Tensor, want_q: bool = True, want_qt: bool = Fals
             qt = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
             st = colmajor_grid(cb, rb, x.device)
         qtp, stp, ldqt, ldst = qt.data_ptr(), st.data_ptr(), qt.stride(0), _grid_ld(st, cb)
-    _check("fp8_quant_128x128", lib().fp8_quant_128x128(x.data_ptr(), xt, rows, cols, _ld(x), qp, ldq, sp, lds,
-                                                        qtp, ldqt, stp, ldst, _stream(x)))
+    args = (x.data_ptr(), xt, rows, cols, _ld(x), qp, ldq, sp, lds, qtp, ldqt, stp, ldst)
+    if rule == SCALE_RULE_FP32:
+        _check("fp8_quant_128x128", lib().fp8_quant_128x128(*args, _stream(x)))
+    else:
+        _check("fp8_quant_128x128_ex", lib().fp8_quant_128x128_ex(*args, int(rule), _stream(x)))
     return q, s, qt, st
 
 
@@ -233,7 +257,7 @@ def fp8_scaled_gemm(A: torch.Tensor, Bt: torch.Tensor, scale_a: torch.Tensor, sc
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A.device)
     oc = F32 if out.dtype == torch.float32 else BF16
-    if mode in (SCALE_BLOCK_1x128_128x128, SCALE_BLOCK_1x128_1x128):
+    if mode in BLOCK_MODES:
         ld_sa = _grid_ld(scale_a, M)
         ld_sb = _grid_ld(scale_b, scale_b.shape[0])
     else:
@@ -268,7 +292,7 @@ def fp8_scaled_gemm_ex(A: torch.Tensor, B: torch.Tensor, b_major: int, scale_a: 
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A.device)
     oc = F32 if out.dtype == torch.float32 else BF16
-    if mode in (SCALE_BLOCK_1x128_128x128, SCALE_BLOCK_1x128_1x128):
+    if mode in BLOCK_MODES:
         ld_sa = _grid_ld(scale_a, M)
         ld_sb = _grid_ld(scale_b, scale_b.shape[0])
     else:

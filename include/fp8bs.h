@@ -51,7 +51,9 @@ typedef enum {
     FP8BS_ERR_WORKSPACE = 4,     /* workspace given but smaller than required           */
     FP8BS_ERR_CUDA = 5,          /* a CUDA runtime/driver call or launch failed         */
     FP8BS_ERR_TIMEOUT = 6,       /* a device-side wait ran past its limit (see below)   */
-    FP8BS_ERR_NO_SM100 = 7       /* current device is not compute capability 10.x     */
+    FP8BS_ERR_NO_SM100 = 7,      /* current device is not compute capability 10.x     */
+    FP8BS_ERR_SCALE = 8          /* a power-of-two GEMM recipe met a scale that is not an
+                                    exact power of two (device-side, see below)          */
 } fp8bs_status;
 
 typedef enum { FP8BS_BF16 = 0, FP8BS_F32 = 1 } fp8bs_dtype;
@@ -60,10 +62,22 @@ typedef enum {
     FP8BS_SCALE_TENSOR = 0,              /* rA = scale_a[0],              rB = scale_b[0]               */
     FP8BS_SCALE_ROWWISE = 1,             /* rA = scale_a[m],              rB = scale_b[n]               */
     FP8BS_SCALE_BLOCK_1x128_128x128 = 2, /* rA = scale_a[m + kb*ld_sa],   rB = scale_b[n/128 + kb*ld_sb] */
-    FP8BS_SCALE_BLOCK_1x128_1x128 = 3    /* rA = scale_a[m + kb*ld_sa],   rB = scale_b[n + kb*ld_sb]     */
+    FP8BS_SCALE_BLOCK_1x128_1x128 = 3,   /* rA = scale_a[m + kb*ld_sa],   rB = scale_b[n + kb*ld_sb]     */
+    /* The same two block recipes with power-of-two scales, applied by the
+     * tensor cores' block-scaled MMA (see fp8_scaled_gemm). */
+    FP8BS_SCALE_BLOCK_1x128_128x128_POW2 = 4,
+    FP8BS_SCALE_BLOCK_1x128_1x128_POW2 = 5
 } fp8bs_scale_mode;
 
 typedef enum { FP8BS_SCALE_COL_MAJOR = 0 } fp8bs_scale_layout;
+
+/* The scale rule of the group quantizations (the *_ex entry points).
+ * FP32: s = 448 / max(amax, 1e-12) in fp32, the rule of every other entry point.
+ * POW2: s = the largest power of two not above that fp32 value, so that the
+ *       stored reciprocal 1/s is an exact power of two: the form a UE8M0 scale
+ *       factor (8-bit biased exponent) holds, which the POW2 GEMM recipes
+ *       take.  q = e4m3(x * s) and the stored 1/s as for FP32. */
+typedef enum { FP8BS_SCALE_RULE_FP32 = 0, FP8BS_SCALE_RULE_POW2 = 1 } fp8bs_scale_rule;
 
 /*
  * fp8_quant_1x128 -- dynamic quantization with one scale per 1x128 group.
@@ -155,6 +169,30 @@ fp8bs_status fp8_quant_128x128(const void* x, fp8bs_dtype xt, int64_t rows, int6
                                uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale,
                                uint8_t* q_t, int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t,
                                cudaStream_t stream);
+
+/*
+ * fp8_quant_1x128_ex, fp8_quant_1x128_dual_ex, fp8_quant_128x128_ex -- the
+ * three group quantizations above with a selectable scale rule.
+ *
+ * Defined by: the entry points without the suffix (same arguments, layouts,
+ * alignment rules and errors) and the scale rule `rule` (fp8bs_scale_rule):
+ * FP8BS_SCALE_RULE_FP32 gives byte-identical results to them;
+ * FP8BS_SCALE_RULE_POW2 rounds each group's fp32 scale down to a power of two
+ * before quantizing, for the power-of-two GEMM recipes (the fast-accumulation
+ * variant of pytorch/pytorch issue #159940, Describe the bug: USE_FAST_ACCUM,
+ * in its B200 form).  An unknown rule gives FP8BS_ERR_UNSUPPORTED.
+ */
+fp8bs_status fp8_quant_1x128_ex(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                                uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale,
+                                int transpose_out, fp8bs_scale_rule rule, cudaStream_t stream);
+fp8bs_status fp8_quant_1x128_dual_ex(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                                     uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale,
+                                     uint8_t* q_t, int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t,
+                                     fp8bs_scale_rule rule, cudaStream_t stream);
+fp8bs_status fp8_quant_128x128_ex(const void* x, fp8bs_dtype xt, int64_t rows, int64_t cols, int64_t ldx,
+                                  uint8_t* q, int64_t ldq, float* scale_inv, int64_t ld_scale,
+                                  uint8_t* q_t, int64_t ldq_t, float* scale_inv_t, int64_t ld_scale_t,
+                                  fp8bs_scale_rule rule, cudaStream_t stream);
 
 /*
  * fp8_quant_tensor -- dynamic quantization with one scale for the whole tensor.
@@ -250,6 +288,19 @@ fp8bs_status fp8_quant_rowwise(const void* x, fp8bs_dtype xt, int64_t rows, int6
  * element size.  Any ldd >= N works; when D is 16-byte aligned and
  * ldd*sizeof(out) is a multiple of 16 the output is written in 16-byte
  * chunks, otherwise element by element.
+ *
+ * The power-of-two recipes BLOCK_1x128_128x128_POW2 and BLOCK_1x128_1x128_POW2
+ * compute the same sum with the scale grids of their plain counterparts, but
+ * every scale must be an exact power of two in [2^-126, 2^127] (what
+ * fp8_quant_*_ex with FP8BS_SCALE_RULE_POW2 writes).  The tensor cores apply
+ * the scales (block-scaled MMA with UE8M0 scale factors, each 128-wide K block
+ * given as four identical 32-wide blocks) and accumulate every K block of a
+ * tile (of a split, with split-K) in one fp32 accumulator, without the
+ * per-K-block promotion in registers: the fast-accumulation variant of
+ * pytorch/pytorch issue #159940 (Describe the bug: USE_FAST_ACCUM), in its
+ * B200 form.  A scale that is not such a power of two sets the device error
+ * flag (fp8bs_check_device_error returns FP8BS_ERR_SCALE) and the output is
+ * unspecified.
  */
 size_t fp8_scaled_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp8bs_scale_mode mode);
 fp8bs_status fp8_scaled_gemm(int64_t M, int64_t N, int64_t K,
@@ -285,7 +336,8 @@ typedef enum {
  *            order, ceil(K/128) x ceil(N/128): rB(n, kb) = scale_b[kb + (n/128)*ld_sb],
  *            ld_sb >= ceil(K/128) (as fp8_quant_128x128 writes it for the K x N
  *            matrix).
- *            BLOCK_1x128_1x128: FP8BS_ERR_UNSUPPORTED.
+ *            BLOCK_1x128_1x128 and the POW2 recipes with B_MN: FP8BS_ERR_UNSUPPORTED
+ *            (with FP8BS_MAJOR_K every recipe is fp8_scaled_gemm's).
  * Everything else (A, scale_a, D, workspace, alignment, errors) as
  * fp8_scaled_gemm.  Asynchronous on `stream`.
  */
@@ -316,7 +368,7 @@ fp8bs_status fp8_scaled_gemm_ex(int64_t M, int64_t N, int64_t K,
  * scale_out  grid M x ceil(N/128) of reciprocal scales, scale_out[m + g*ld_scale_out],
  *            ld_scale_out >= M, ld_scale_out % 4 == 0.
  * q_out and scale_out 16-byte aligned.  The caller owns every buffer.
- * Recipes: TENSOR, ROWWISE and BLOCK_1x128_128x128; BLOCK_1x128_1x128 returns
+ * Recipes: TENSOR, ROWWISE and BLOCK_1x128_128x128; the others return
  * FP8BS_ERR_UNSUPPORTED.  Errors as fp8_scaled_gemm; nothing is launched when
  * a check fails.  Asynchronous on `stream`.
  */
@@ -368,7 +420,9 @@ const char* fp8bs_status_string(fp8bs_status s);
  * internal pipeline barriers (a few seconds); a wait that runs out sets the
  * flag, the kernel drains its copies in flight, frees its tensor memory and
  * returns, so the CUDA context stays usable.  Returns FP8BS_ERR_TIMEOUT if the
- * flag was set, FP8BS_ERR_CUDA if the stream reports an error, else FP8BS_OK.
+ * flag was set by a wait, FP8BS_ERR_SCALE if it was set only by a power-of-two
+ * GEMM recipe that met a scale which is not a power of two, FP8BS_ERR_CUDA if
+ * the stream reports an error, else FP8BS_OK.
  */
 fp8bs_status fp8bs_check_device_error(cudaStream_t stream);
 

@@ -15,6 +15,9 @@ only the named kernel runs R times):
   gemm_fwd_then_quant  the forward GEMM, then fp8_quant_1x128 of its output (two launches)
   gemm_longk   256 x 512 x 128128 (k_blocks 1001), 1x128 x 128x128, split-K, bf16 out
   gemm_longk_mn        the same with x (K x 512) quantized as stored and read MN-major
+  gemm_longk_1x128     the long-K GEMM with the 1x128 x 1x128 recipe
+  <gemm case>_pow2     gemm_fwd, gemm_dgrad_wt, gemm_wgrad, gemm_longk, gemm_longk_1x128 with
+                       power-of-two scales on the block-scaled MMA (the fast-accumulation variant)
   gemm_grouped         grouped GEMM: 8 groups x 2080 tokens over (N, K) = (5120, 8192), 1x128 x 128x128
   gemm_grouped_ragged  the same with ragged group sizes (4000, 1, 127, 129, 3000, 0, 5000, 4383)
   quant_rows   1x128 quantization of a 32768 x 32768 bf16 matrix
@@ -42,8 +45,19 @@ import torch
 from fp8_block_scaled_11_b200 import inputs, ops
 
 
+# block recipe -> the same recipe with power-of-two scales (block-scaled MMA)
+_POW2_MODE = {ops.SCALE_BLOCK_1x128_128x128: ops.SCALE_BLOCK_1x128_128x128_POW2,
+              ops.SCALE_BLOCK_1x128_1x128: ops.SCALE_BLOCK_1x128_1x128_POW2}
+
+
 def _gemm_case(name):
     M = inputs.LLAMA4_M
+    # "<case>_pow2": the case's operands quantized with the power-of-two rule,
+    # multiplied by the power-of-two recipe
+    pow2 = name.endswith("_pow2")
+    if pow2:
+        name = name[:-len("_pow2")]
+    R = ops.SCALE_RULE_POW2 if pow2 else ops.SCALE_RULE_FP32
     if name == "gemm_tiny":
         A, Bt = inputs.tiny_blockwise()
         qa, sa = ops.fp8_quant_1x128(A.cuda())
@@ -66,8 +80,8 @@ def _gemm_case(name):
         x, W, _ = inputs.llama4(5120, 8192)
         x, W = x.cuda(), W.cuda()
         if name == "gemm_fwd":
-            qa, sa = ops.fp8_quant_1x128(x)
-            qb, sb, _, _ = ops.fp8_quant_128x128(W)
+            qa, sa = ops.fp8_quant_1x128(x, rule=R)
+            qb, sb, _, _ = ops.fp8_quant_128x128(W, rule=R)
             mode = ops.SCALE_BLOCK_1x128_128x128
         elif name == "gemm_rowwise":
             (qa, sa), (qb, sb) = ops.fp8_quant_rowwise(x), ops.fp8_quant_rowwise(W)
@@ -80,7 +94,7 @@ def _gemm_case(name):
         flops = 2.0 * M * 5120 * 8192
     elif name in ("gemm_dgrad", "gemm_dgrad_wt"):
         _, W, dy = inputs.llama4(5120, 8192)
-        qa, sa = ops.fp8_quant_1x128(dy.cuda())
+        qa, sa = ops.fp8_quant_1x128(dy.cuda(), rule=R)
         mode = ops.SCALE_BLOCK_1x128_128x128
         out = torch.empty((M, 8192), dtype=torch.bfloat16, device="cuda")
         flops = 2.0 * M * 8192 * 5120
@@ -89,11 +103,11 @@ def _gemm_case(name):
             qw, sw, _, _ = ops.fp8_quant_128x128(W.cuda())
             torch.cuda.synchronize()
             return (lambda: ops.fp8_scaled_gemm_ex(qa, qw, ops.MAJOR_MN, sa, sw, mode, out=out)), flops, "TFLOP/s"
-        _, _, qb, sb = ops.fp8_quant_128x128(W.cuda(), want_q=False, want_qt=True)
+        _, _, qb, sb = ops.fp8_quant_128x128(W.cuda(), want_q=False, want_qt=True, rule=R)
     elif name == "gemm_wgrad":
         x, _, dy = inputs.llama4(5120, 8192)
-        qa, sa = ops.fp8_quant_1x128(dy.cuda(), transpose_out=True)
-        qb, sb = ops.fp8_quant_1x128(x.cuda(), transpose_out=True)
+        qa, sa = ops.fp8_quant_1x128(dy.cuda(), transpose_out=True, rule=R)
+        qb, sb = ops.fp8_quant_1x128(x.cuda(), transpose_out=True, rule=R)
         mode = ops.SCALE_BLOCK_1x128_1x128
         out = torch.empty((5120, 8192), dtype=torch.bfloat16, device="cuda")
         flops = 2.0 * M * 5120 * 8192
@@ -110,13 +124,22 @@ def _gemm_case(name):
         torch.cuda.synchronize()
         return (lambda: ops.fp8_scaled_gemm_ex(qa, qb, ops.MAJOR_MN, sa, sb, mode, out=out, workspace=wsb)), flops, \
             "TFLOP/s"
+    elif name == "gemm_longk_1x128":
+        goT, x = inputs.long_k(128128)
+        qa, sa = ops.fp8_quant_1x128(goT.cuda(), rule=R)
+        qb, sb = ops.fp8_quant_1x128(x.cuda(), transpose_out=True, rule=R)
+        mode = ops.SCALE_BLOCK_1x128_1x128
+        out = torch.empty((256, 512), dtype=torch.bfloat16, device="cuda")
+        flops = 2.0 * 256 * 512 * 128128
     else:
         goT, x = inputs.long_k(128128)
-        qa, sa = ops.fp8_quant_1x128(goT.cuda())
-        _, _, qb, sb = ops.fp8_quant_128x128(x.cuda(), want_q=False, want_qt=True)
+        qa, sa = ops.fp8_quant_1x128(goT.cuda(), rule=R)
+        _, _, qb, sb = ops.fp8_quant_128x128(x.cuda(), want_q=False, want_qt=True, rule=R)
         mode = ops.SCALE_BLOCK_1x128_128x128
         out = torch.empty((256, 512), dtype=torch.bfloat16, device="cuda")
         flops = 2.0 * 256 * 512 * 128128
+    if pow2:
+        mode = _POW2_MODE[mode]
     ws = ops.fp8_scaled_gemm_workspace_size(qa.shape[0], qb.shape[0], qa.shape[1], mode)
     wsb = torch.empty((max(ws, 16),), dtype=torch.uint8, device="cuda")
     torch.cuda.synchronize()
@@ -206,7 +229,8 @@ def _quant_case(name):
 CONFIG_CASES = (["gemm_tiny", "gemm_pertensor_small", "gemm_rowwise_small", "gemm_fwd", "gemm_dgrad", "gemm_dgrad_wt",
                  "gemm_wgrad", "gemm_tensor", "gemm_rowwise", "gemm_longk", "gemm_fwd_then_quant",
                  "gemm_fwd_quant", "gemm_fwd_quant_only", "gemm_longk_mn", "gemm_grouped", "gemm_grouped_ragged",
-                 "quant_dual"]
+                 "gemm_longk_1x128", "gemm_fwd_pow2", "gemm_dgrad_wt_pow2", "gemm_wgrad_pow2", "gemm_longk_pow2",
+                 "gemm_longk_1x128_pow2", "quant_dual"]
                 + [f"quant_rows_{n}" for n in inputs.QUANT_SWEEP_SIZES]
                 + [f"quant_tile_{n}" for n in inputs.QUANT_SWEEP_SIZES])
 

@@ -160,3 +160,40 @@ def test_gemm_quant_validation(L):
     assert gq(L, A=0) == INVALID
     assert gq(L, D=GOOD, ldd=100) == INVALID        # stored output with ldd < N
 
+
+
+def test_quant_ex_validation(L):
+    """The scale-rule entry points: an unknown rule is refused; with a known
+    rule they validate exactly as the plain entry points."""
+    f = L.fp8_quant_1x128_ex
+    assert f(GOOD, 0, 256, 256, 256, GOOD, 256, GOOD, 256, 0, 2, None) == UNSUPPORTED
+    for rule in (0, 1):
+        assert f(0, 0, 256, 256, 256, GOOD, 256, GOOD, 256, 0, rule, None) == INVALID
+        assert f(GOOD, 0, 256, 256, 256, GOOD, 256, GOOD, 258, 0, rule, None) == ALIGN
+        assert f(GOOD, 0, 256, 256, 256, GOOD, 256, GOOD, 100, 0, rule, None) == INVALID
+    d = L.fp8_quant_1x128_dual_ex
+    assert d(GOOD, 0, 256, 384, 384, GOOD, 384, GOOD, 256, GOOD, 256, GOOD, 384, 5, None) == UNSUPPORTED
+    assert d(GOOD, 0, 256, 384, 384, GOOD, 384, GOOD, 256, 0, 256, GOOD, 384, 1, None) == INVALID
+    assert d(GOOD, 0, 256, 384, 384, GOOD, 392, GOOD, 256, GOOD, 256, GOOD, 384, 1, None) == ALIGN
+    t = L.fp8_quant_128x128_ex
+    assert t(GOOD, 0, 256, 256, 256, GOOD, 256, GOOD, 4, 0, 0, 0, 0, -1, None) == UNSUPPORTED
+    assert t(GOOD, 0, 256, 256, 256, 0, 0, 0, 0, 0, 0, 0, 0, 1, None) == INVALID
+    assert t(GOOD, 0, 256, 256, 256, GOOD, 256, GOOD, 2, 0, 0, 0, 0, 1, None) == ALIGN
+
+
+def test_gemm_pow2_validation(L):
+    """The power-of-two recipes take the block recipes' scale grids and their
+    checks; they have no MN-major, fused-quantization or grouped form."""
+    assert gemm(L, mode=4, ldsb=1) == INVALID            # 128x128 grid: ld_sb < ceil(N/128)
+    assert gemm(L, mode=5, ldsb=128) == INVALID          # 1x128 grid: ld_sb < N
+    assert gemm(L, mode=4, ldsa=128) == INVALID          # ld_sa < M
+    assert gemm(L, mode=5, ldsb=258) == ALIGN
+    assert gemm(L, mode=6) == UNSUPPORTED
+    ex = L.fp8_scaled_gemm_ex
+    assert ex(256, 256, 256, GOOD, 256, GOOD, 256, 1, GOOD, 256, GOOD, 4, 4, 0, GOOD, 256, 0, 0, 0, None) == UNSUPPORTED
+    assert gq(L, mode=4) == UNSUPPORTED
+    assert gq(L, mode=5, lsb=384) == UNSUPPORTED
+    # split-K workspace: the power-of-two recipes plan 128 x 256 single-CTA tiles
+    assert L.fp8_scaled_gemm_workspace_size(16640, 5120, 8192, 4) == 0
+    ws = L.fp8_scaled_gemm_workspace_size(256, 512, 128128, 4)
+    assert ws > 0 and ws % 16 == 0
