@@ -269,6 +269,12 @@ def run_gpu(args):
     if not args.no_e2e:
         e2e = run_e2e(args, world, steps, shapes, data, flops_step, barrier)
 
+    # ---- the fast-accumulation ablation: the same step with power-of-two
+    # scales on the block-scaled MMA (no per-K-block promotion)
+    abl = None
+    if not args.no_ablation:
+        abl = run_ablation(args, world, dev_data, shapes, barrier, ms_step, per_gemm_ms)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_sample(args.cpu_rows)
@@ -306,6 +312,7 @@ def run_gpu(args):
         },
         "roofline_gemms": gemm_list,
         "sustained": sus,
+        "fast_accum_ablation": abl,
         "clocks": clocks,
         "gpu_launches": Fp8LinearStep.LAUNCHES_PER_STEP * len(steps) * args.steps,
         "e2e": e2e,
@@ -348,6 +355,60 @@ def gemm_roofline_list(steps, per_gemm_ms, nsteps, fp8_peak, traffic):
                         "algorithmic_bytes": gemm_algorithmic_bytes(M, N, K, recipe),
                         "traffic": traffic.get(key)})
     return out
+
+
+def run_ablation(args, world, dev_data, shapes, barrier, promoted_ms_step, promoted_gemm_ms):
+    """The step with every scale rounded down to a power of two and the GEMMs
+    on the block-scaled MMA (whole-K fp32 accumulation in TMEM): W warm-up
+    and K timed steps with per-GEMM CUDA events, as the main measurement.
+    The accuracy side of the ablation is the parity tests' (against the oracle
+    with the same power-of-two rule)."""
+    import torch
+    from fp8_block_scaled_11_b200 import inputs, ops
+    from fp8_block_scaled_11_b200.linear import Fp8LinearStep
+
+    M = inputs.LLAMA4_M
+    steps = [Fp8LinearStep(M, N, K, pow2=True) for N, K in shapes]
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        for st, (x, W, dy) in zip(steps, dev_data):
+            st.run(x, W, dy)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    events = []
+    t0.record(stream)
+    for _ in range(args.steps):
+        for st, (x, W, dy) in zip(steps, dev_data):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            st.quantize(x, W, dy)
+            st.gemms(mark=lambda i: e[i].record(stream))
+            events.append((st, e))
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    st_err = ops.fp8bs_check_device_error()
+    if st_err != 0:
+        raise SystemExit(f"device error in the ablation: {ops.fp8bs_status_string(st_err)}")
+    per_gemm = [sum(e[g].elapsed_time(e[g + 1]) for st, e in events if st is steps[i])
+                for i in range(len(steps)) for g in range(3)]
+    vals = max_over_ranks([t0.elapsed_time(t1)] + per_gemm, world, "cuda")
+    ms_step = vals[0] / args.steps
+    per_gemm = vals[1:]
+    flops_step = sum(st.flops() for st in steps)
+    names = [f"{GEMM_NAMES[g]} {M_}x{N_}x{K_}" for st in steps
+             for g, (M_, N_, K_, _) in enumerate(gemm_shapes(st))]
+    return {
+        "recipe": "the step's recipes with power-of-two (UE8M0) scales: tcgen05.mma kind::mxf8f6f4.block_scale, "
+                  "whole-K fp32 accumulation in TMEM, no per-K-block promotion (gemm_fp8_bs_kernel)",
+        "ms_per_step": round(ms_step, 4),
+        "value": round(world * flops_step / (ms_step * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "step_speedup_vs_promoted": round(promoted_ms_step / ms_step, 3),
+        "gemm_us": {n: round(v * 1e3 / args.steps, 1) for n, v in zip(names, per_gemm)},
+        "gemm_speedup_vs_promoted": {n: round(a / b, 3) for n, a, b in zip(names, promoted_gemm_ms, per_gemm)},
+    }
 
 
 def run_sustained(args, world, local, one_step, steps, flops_step, peaks, barrier):
@@ -665,6 +726,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ablation", action="store_true",
+                    help="skip the fast-accumulation ablation (power-of-two scales, block-scaled MMA)")
     ap.add_argument("--sustained-s", type=float, default=3.0,
                     help="seconds of back-to-back steps for the sustained-clock figure (0: skip)")
     ap.add_argument("--oracle-configs", action="store_true",

@@ -16,6 +16,11 @@ transposed copy, dy in both directions from one read -- and three GEMM
 launches.  With ``dgrad_wt_copy=False`` W is quantized once and dgrad reads
 the forward's W_q in its stored orientation (B MN-major, fp8_scaled_gemm_ex):
 the same result without the transposed copy, on the CTA-pair GEMM kernel.
+With ``pow2=True`` every quantization uses the power-of-two scale rule and
+the GEMMs the matching power-of-two recipes on the block-scaled MMA (whole-K
+accumulation in TMEM, no per-K-block promotion): the fast-accumulation
+variant of pytorch/pytorch issue #159940 (Describe the bug: USE_FAST_ACCUM)
+in its B200 form, for the speed / accuracy ablation.
 """
 from __future__ import annotations
 
@@ -29,9 +34,15 @@ class Fp8LinearStep:
 
     LAUNCHES_PER_STEP = 6
 
-    def __init__(self, M: int, N: int, K: int, device="cuda", dgrad_wt_copy: bool = True):
+    def __init__(self, M: int, N: int, K: int, device="cuda", dgrad_wt_copy: bool = True, pow2: bool = False):
         self.M, self.N, self.K = M, N, K
+        if pow2 and not dgrad_wt_copy:
+            raise ValueError("the power-of-two recipes read K-major operands only (dgrad_wt_copy=True)")
         self.dgrad_wt_copy = dgrad_wt_copy
+        self.pow2 = pow2
+        self.rule = ops.SCALE_RULE_POW2 if pow2 else ops.SCALE_RULE_FP32
+        self.modes = ((ops.SCALE_BLOCK_1x128_128x128_POW2, ops.SCALE_BLOCK_1x128_1x128_POW2) if pow2
+                      else (ops.SCALE_BLOCK_1x128_128x128, ops.SCALE_BLOCK_1x128_1x128))
         d = device
         u8 = torch.uint8
         g = ops.colmajor_grid
@@ -51,21 +62,21 @@ class Fp8LinearStep:
         self.y = torch.empty((M, N), dtype=bf, device=d)
         self.dx = torch.empty((M, K), dtype=bf, device=d)
         self.dW = torch.empty((N, K), dtype=bf, device=d)
-        ws = max(ops.fp8_scaled_gemm_workspace_size(M, N, K, ops.SCALE_BLOCK_1x128_128x128),
-                 ops.fp8_scaled_gemm_workspace_size(M, K, N, ops.SCALE_BLOCK_1x128_128x128),
-                 ops.fp8_scaled_gemm_workspace_size(N, K, M, ops.SCALE_BLOCK_1x128_1x128))
+        ws = max(ops.fp8_scaled_gemm_workspace_size(M, N, K, self.modes[0]),
+                 ops.fp8_scaled_gemm_workspace_size(M, K, N, self.modes[0]),
+                 ops.fp8_scaled_gemm_workspace_size(N, K, M, self.modes[1]))
         self.workspace = torch.empty((max(ws, 16),), dtype=u8, device=d)
 
     def quantize(self, x: torch.Tensor, W: torch.Tensor, dy: torch.Tensor):
-        ops.fp8_quant_1x128_dual(x, out=(self.xq, self.xs, self.xtq, self.xts))
+        ops.fp8_quant_1x128_dual(x, out=(self.xq, self.xs, self.xtq, self.xts), rule=self.rule)
         ops.fp8_quant_128x128(W, want_q=True, want_qt=self.dgrad_wt_copy,
-                              out=(self.wq, self.ws, self.wtq, self.wts))
-        ops.fp8_quant_1x128_dual(dy, out=(self.dyq, self.dys, self.dytq, self.dyts))
+                              out=(self.wq, self.ws, self.wtq, self.wts), rule=self.rule)
+        ops.fp8_quant_1x128_dual(dy, out=(self.dyq, self.dys, self.dytq, self.dyts), rule=self.rule)
 
     def gemms(self, mark=None):
         """The three GEMMs; `mark(i)` (optional) is called before GEMM i and
         after the last one (i = 3), e.g. to record CUDA events between them."""
-        B2, B3 = ops.SCALE_BLOCK_1x128_128x128, ops.SCALE_BLOCK_1x128_1x128
+        B2, B3 = self.modes
         mark = mark or (lambda i: None)
         mark(0)
         ops.fp8_scaled_gemm(self.xq, self.wq, self.xs, self.ws, B2, out=self.y, workspace=self.workspace)

@@ -269,3 +269,31 @@ def test_gemm_pow2_unsupported_forms():
         ops.fp8_scaled_gemm_ex(A, A, ops.MAJOR_MN, s, sb, ops.SCALE_BLOCK_1x128_128x128_POW2)
     with pytest.raises(ops.Fp8bsError):
         ops.fp8_scaled_gemm_quant(A, A, s, sb, ops.SCALE_BLOCK_1x128_128x128_POW2)
+
+
+@pytest.mark.parametrize("K", [8192, 32768, 128128])
+def test_whole_k_accumulation_error_bound(K):
+    """The accuracy cost of the fast-accumulation variant: one unit's whole K
+    range accumulated in TMEM (split-K off) loses at most about one fp32 unit
+    roundoff per 32-wide MMA step, relative Frobenius error <= (K/32) * 2^-23
+    against the oracle, while the promoted recipe on the same power-of-two
+    operands stays within the method's 1e-5."""
+    rng = np.random.default_rng(K)
+    M, N = 256, 512
+    Kb = (K + 127) // 128
+    A = inputs.random_e4m3_bytes(M, K, seed=1)
+    B = inputs.random_e4m3_bytes(N, K, seed=2)
+    sa, sb = pow2_scales(rng, (M, Kb)), pow2_scales(rng, ((N + 127) // 128, Kb))
+    rows = [0, 1, 100, 255]
+    ref = oracle.gemm(A.numpy(), B.numpy(), sa, sb, ops.SCALE_BLOCK_1x128_128x128, rows=rows)
+    r = torch.as_tensor(rows, device="cuda")
+    Ad, Bd = A.cuda(), B.cuda()
+    fast = ops.fp8_scaled_gemm(Ad, Bd, to_grid(sa), to_grid(sb), ops.SCALE_BLOCK_1x128_128x128_POW2,
+                               out_dtype=torch.float32, split_k=False)
+    prom = ops.fp8_scaled_gemm(Ad, Bd, to_grid(sa), to_grid(sb), ops.SCALE_BLOCK_1x128_128x128,
+                               out_dtype=torch.float32, split_k=False)
+    torch.cuda.synchronize()
+    no_device_error()
+    rel = lambda D: np.linalg.norm(D[r].double().cpu().numpy() - ref) / np.linalg.norm(ref)
+    assert rel(fast) <= (K / 32) * 2.0 ** -23, rel(fast)
+    assert rel(prom) <= 1e-5, rel(prom)
