@@ -15,23 +15,29 @@
 // skipped here too, at the price of scales restricted to powers of two.
 //
 // One persistent CTA per SM computes 128 x 256 output tiles (units: tiles, or
-// tile x K-split with split-K), 16 warps:
+// tile x K-split with split-K), 12 warps:
 //   warp 0      TMA producer: per K-block a 128x128 tile of A and a 256x128
 //               tile of B^T (128-byte swizzle) into a 4-stage ring.
-//   warp 1      TMEM allocation; lane 0 issues four 128x256x32 block-scaled
+//   warp 1      TMEM allocation; lane 0, per group of four K-blocks, copies
+//               the group's scale factors from shared memory into a stage of
+//               the TMEM scale-factor ring (columns 256..) with three
+//               tcgen05.cp 32x128b.warpx4 (every lane quarter gets its copy,
+//               as the MMA reads it), then issues four 128x256x32 block-scaled
 //               MMAs per K-block into the accumulator (TMEM columns 0..255).
 //   warp 2      scale producer: per group of four K-blocks one TMA load of the
 //               A scale grid's 128 x 4 block and one of B's (256 x 4, or the
 //               aligned 4 x 4 group of 128-column blocks) into a shared-memory
 //               scale ring, running up to four groups ahead.
-//   warps 4-7   scale-factor writers, one per TMEM sub-partition: per group of
-//               four K-blocks they read the fp32 scales from the scale ring,
-//               take each one's exponent byte and tcgen05.st one 16-column
-//               stage of the scale-factor ring (columns 256..); every
-//               sub-partition holds its own copy, as the MMA reads it.
-//   warps 8-15  epilogue: load the finished accumulator into registers
+//   warp 3      scale-factor converter: per group it reads the fp32 scales,
+//               takes each one's exponent byte and writes the bytes in the
+//               TMEM layout (one 16-byte row per lane) into a staging ring.
+//   warps 4-11  epilogue: load the finished accumulator into registers
 //               (128 columns per thread), release it to the next unit's MMAs,
 //               then convert and store.
+// The scale-factor work stays on the first warpgroup: a first form with four
+// writer warps (one per lane quarter, tcgen05.st) cost the MMA ~70 us of
+// 630 on the Llama4 forward GEMM by sharing every SM sub-partition with the
+// MMA and TMA threads.
 // Scale-factor layout in TMEM (M = 128, N = 256, one CTA, one factor per 32
 // K): the factor of row r (of A, or of B^T) sits in lane 32*q + r % 32 for
 // each sub-partition q, in 32-bit column r / 32 of the operand's part of the
@@ -61,34 +67,31 @@ constexpr uint32_t kSfCols = 16;                // TMEM columns per stage
 constexpr uint32_t kSfColA = 0;                 // A's 4 words (128 rows / 32) within a stage
 constexpr uint32_t kSfColB = 8;                 // B's 8 words (256 columns / 32)
 constexpr uint32_t kSfCol0 = kBN;               // the ring follows the accumulator
-constexpr int kBsThreads = 512;
 constexpr int kBsEpiWarps = 8;
-constexpr int kBsSfWarps = 4;
-// register hand-over (setmaxnreg) from the 128 per thread of the launch:
-// control warpgroup 40, scale-factor writers 88, epilogue 192
-constexpr int kBsLaunchRegs = 65536 / kBsThreads;
-constexpr int kBsCtrlRegs = 40;
-constexpr int kBsSfRegs = 88;
-constexpr int kBsEpiRegs = 192;
-static_assert(128 * kBsCtrlRegs + 128 * kBsSfRegs + 32 * kBsEpiWarps * kBsEpiRegs <= kBsThreads * kBsLaunchRegs,
-              "register hand-over exceeds the launch allocation");
+constexpr int kBsThreads = 32 * (4 + kBsEpiWarps);
 static_assert(kSfCol0 + kSfStages * kSfCols <= kTmemCols, "scale-factor ring exceeds TMEM");
 
 // one scale-ring stage: A's scales [b][128 rows], then B's [b][256 columns]
 // (or [b][4 blocks]), b = the stage's four K-blocks
 constexpr uint32_t kScStageBytes = (kBM + kBN) * kSfKb * 4;
+// one staging stage of scale-factor bytes, each part 32 rows of 16 bytes (the
+// source of one tcgen05.cp 32x128b): A, then B's columns 0..127, then 128..255
+constexpr uint32_t kSfPartBytes = 32 * 16;
+constexpr uint32_t kSfStageBytes = 3 * kSfPartBytes;
 
 struct BsSmem {
     static constexpr uint32_t a_off = 0;
     static constexpr uint32_t b_off = a_off + kBsStages * kATileBytes;
     static constexpr uint32_t sc_off = b_off + kBsStages * kBTileBytes;
-    static constexpr uint32_t bar_off = sc_off + kSfStages * kScStageBytes;
+    static constexpr uint32_t sf_off = sc_off + kSfStages * kScStageBytes;
+    static constexpr uint32_t bar_off = sf_off + kSfStages * kSfStageBytes;
     // ab_full[S], ab_empty[S], sf_full[SS], sf_empty[SS], sc_full[SS], sc_empty[SS], tm_full, tm_empty, drain
     static constexpr uint32_t n_bars = 2 * kBsStages + 4 * kSfStages + 3;
     static constexpr uint32_t misc_off = bar_off + n_bars * 8;
     static constexpr uint32_t total = misc_off + 16;
     static constexpr uint32_t alloc = total + 1024;     // slack to align the base to 1024 B
 };
+static_assert(BsSmem::alloc <= 232448, "shared memory per CTA");
 
 // The UE8M0 byte of a power-of-two scale r = 2^(e-127): its fp32 biased
 // exponent.  Anything else (a mantissa bit, the sign, zero or subnormal,
@@ -133,10 +136,10 @@ gemm_fp8_bs_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             mbar_init(ab_empty(s), 1);
         }
         for (int s = 0; s < kSfStages; ++s) {
-            mbar_init(sf_full(s), kBsSfWarps);
+            mbar_init(sf_full(s), 1);
             mbar_init(sf_empty(s), 1);
             mbar_init(sc_full(s), 1);
-            mbar_init(sc_empty(s), kBsSfWarps);
+            mbar_init(sc_empty(s), 1);
         }
         mbar_init(tm_full, 1);
         mbar_init(tm_empty, kBsEpiWarps);
@@ -167,7 +170,6 @@ gemm_fp8_bs_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     };
 
     if (warp < 4) {
-        setmaxnreg_dec<kBsCtrlRegs>();
         if (warp == 0) {
             // ------------------------------------------------------------ producer
             if (lane == 0) {
@@ -211,6 +213,13 @@ gemm_fp8_bs_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                         if (j == 0 && !mbar_wait_bounded(sf_full(ss), sphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t sf = tmem_base + kSfCol0 + (uint32_t)ss * kSfCols;
+                        if (j == 0) {
+                            // the stage's factors: A's 4 words, B's 8 words (two copies of 4)
+                            const uint32_t src = sbase + BsSmem::sf_off + (uint32_t)ss * kSfStageBytes;
+                            tmem_cp_32x128b_x4(sf + kSfColA, smem_desc_cp_rows16(src));
+                            tmem_cp_32x128b_x4(sf + kSfColB, smem_desc_cp_rows16(src + kSfPartBytes));
+                            tmem_cp_32x128b_x4(sf + kSfColB + 4, smem_desc_cp_rows16(src + 2 * kSfPartBytes));
+                        }
                         const uint32_t sfa = (sf + kSfColA) | (j << 30);
                         const uint32_t sfb = (sf + kSfColB) | (j << 30);
                         const uint32_t idesc = idesc_e4m3_bs(kBM, kBN, j);
@@ -266,82 +275,82 @@ gemm_fp8_bs_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 for (int s = 0; s < kSfStages; ++s)
                     if (filled >> s & 1u) mbar_wait_bounded(sc_full(s), fill_par >> s & 1u, nullptr, kDrainLimitNs);
             }
-        }
-    } else if (warp < 4 + kBsSfWarps) {
-        setmaxnreg_dec<kBsSfRegs>();
-        // ------------------------------------------------------------ scale-factor writers
-        const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-        int ss = 0;
-        uint32_t sphase = 0;
-        bool ok = true;
-        uint32_t bad = 0;
-        for (int64_t u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-            int tm, tn, kb0, kb1, split;
-            decode_unit(p, u, tm, tn, kb0, kb1, split);
-            const int m0 = tm * kBM, n0 = tn * kBN;
-            for (int kbase = kb0; kbase < kb1; kbase += kSfKb) {
-                // every lane waits (the TMEM store below is warp-collective); a
-                // wait that gives up raises the abort flag, the outcome is voted per unit
-                if (!mbar_wait_bounded(sc_full(ss), sphase, abort_flag, kWaitLimitNs)) ok = false;
-                const float* sc = reinterpret_cast<const float*>(smem + BsSmem::sc_off + (uint32_t)ss * kScStageBytes);
-                const float* scb = sc + kBM * kSfKb;
-                uint32_t w[16];
+        } else {
+            // ------------------------------------------------------------ scale-factor converter
+            int ss = 0;
+            uint32_t sphase = 0;
+            bool ok = true;
+            uint32_t bad = 0;
+            for (int64_t u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+                int tm, tn, kb0, kb1, split;
+                decode_unit(p, u, tm, tn, kb0, kb1, split);
+                const int m0 = tm * kBM, n0 = tn * kBN;
+                for (int kbase = kb0; kbase < kb1; kbase += kSfKb) {
+                    // every lane waits; a wait that gives up raises the abort
+                    // flag, the outcome is voted per unit
+                    if (!mbar_wait_bounded(sc_full(ss), sphase, abort_flag, kWaitLimitNs)) ok = false;
+                    const float* sc = reinterpret_cast<const float*>(smem + BsSmem::sc_off + (uint32_t)ss * kScStageBytes);
+                    const float* scb = sc + kBM * kSfKb;
+                    // lane l's 16-byte row of each part: word j = rows (columns) 32j + l,
+                    // byte b = K-block kbase + b
+                    uint32_t wa[4], wb[8];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int m = m0 + 32 * j + lane;
-                    uint32_t word = 0;
+                    for (int j = 0; j < 4; ++j) {
+                        const int m = m0 + 32 * j + lane;
+                        uint32_t word = 0;
 #pragma unroll
-                    for (int b = 0; b < kSfKb; ++b) {
-                        uint32_t e = 127u;                       // 1.0 where no row or K-block is
-                        if (m < p.M && kbase + b < kb1) e = ue8m0_of(sc[b * kBM + 32 * j + lane], bad);
-                        word |= e << (8 * b);
+                        for (int b = 0; b < kSfKb; ++b) {
+                            uint32_t e = 127u;                       // 1.0 where no row or K-block is
+                            if (m < p.M && kbase + b < kb1) e = ue8m0_of(sc[b * kBM + 32 * j + lane], bad);
+                            word |= e << (8 * b);
+                        }
+                        wa[j] = word;
                     }
-                    w[kSfColA + j] = word;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        int idx, col;                                 // global index, index within the ring stage
+                        if (MODE == kModeBlock128) {
+                            idx = (n0 >> 7) + (j >> 2);               // the 128-column block of columns n0+32j ..
+                            col = (idx & 3);
+                        } else {
+                            idx = n0 + 32 * j + lane;
+                            col = 32 * j + lane;
+                        }
+                        const bool valid = MODE == kModeBlock128 ? idx * 128 < p.N : idx < p.N;
+                        constexpr int kBW = MODE == kModeBlock128 ? 4 : kBN;   // B entries per K-block in the stage
+                        uint32_t word = 0;
+#pragma unroll
+                        for (int b = 0; b < kSfKb; ++b) {
+                            uint32_t e = 127u;
+                            if (valid && kbase + b < kb1) e = ue8m0_of(scb[b * kBW + col], bad);
+                            word |= e << (8 * b);
+                        }
+                        wb[j] = word;
+                    }
+                    // the fp32 stage is read: back to the scale producer
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sc_empty(ss));
+                    // the staging stage is free once the MMA thread's copies from it
+                    // (and the MMAs reading the TMEM stage they fill) have completed
+                    if (!mbar_wait_bounded(sf_empty(ss), sphase ^ 1u, abort_flag, kWaitLimitNs)) ok = false;
+                    const uint32_t dst = sbase + BsSmem::sf_off + (uint32_t)ss * kSfStageBytes + (uint32_t)lane * 16u;
+                    sts128(dst, wa[0], wa[1], wa[2], wa[3]);
+                    sts128(dst + kSfPartBytes, wb[0], wb[1], wb[2], wb[3]);
+                    sts128(dst + 2 * kSfPartBytes, wb[4], wb[5], wb[6], wb[7]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sf_full(ss));
+                    if (++ss == kSfStages) { ss = 0; sphase ^= 1u; }
                 }
-#pragma unroll
-                for (int j = 4; j < 8; ++j) w[j] = 0u;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    int idx, col;                                 // global index, index within the ring stage
-                    if (MODE == kModeBlock128) {
-                        idx = (n0 >> 7) + (j >> 2);               // the 128-column block of columns n0+32j ..
-                        col = (idx & 3);
-                    } else {
-                        idx = n0 + 32 * j + lane;
-                        col = 32 * j + lane;
-                    }
-                    const bool valid = MODE == kModeBlock128 ? idx * 128 < p.N : idx < p.N;
-                    constexpr int kBW = MODE == kModeBlock128 ? 4 : kBN;   // B entries per K-block in the stage
-                    uint32_t word = 0;
-#pragma unroll
-                    for (int b = 0; b < kSfKb; ++b) {
-                        uint32_t e = 127u;
-                        if (valid && kbase + b < kb1) e = ue8m0_of(scb[b * kBW + col], bad);
-                        word |= e << (8 * b);
-                    }
-                    w[kSfColB + j] = word;
-                }
-                // the scale stage is read: back to the scale producer
-                __syncwarp();
-                if (lane == 0) mbar_arrive(sc_empty(ss));
-                if (!mbar_wait_bounded(sf_empty(ss), sphase ^ 1u, abort_flag, kWaitLimitNs)) ok = false;
-                tc_fence_after();
-                tmem_st_32x32b_x16(tmem_base + lane_addr + kSfCol0 + (uint32_t)ss * kSfCols, w);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(sf_full(ss));
-                if (++ss == kSfStages) { ss = 0; sphase ^= 1u; }
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
             }
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
+            if (!ok && lane == 0) give_up();
+            if (__any_sync(0xffffffffu, bad != 0) && lane == 0) atomicOr(p.err, 2);
         }
-        if (!ok && lane == 0) give_up();
-        if (__any_sync(0xffffffffu, bad != 0) && lane == 0) atomicOr(p.err, 2);
     } else {
-        setmaxnreg_inc<kBsEpiRegs>();
         // ------------------------------------------------------------ epilogue
-        const int e = warp - 4 - kBsSfWarps;     // 0 .. 7
+        const int e = warp - 4;                  // 0 .. 7
         const int lq = warp & 3;                 // TMEM lane quarter this warp may access
         const int col0 = (e >> 2) * 128;         // this warp's 128 columns of the tile
         const uint32_t taddr = tmem_base + ((uint32_t)(lq * 32) << 16) + (uint32_t)col0;

@@ -1,6 +1,7 @@
 // ptx_bs.cuh -- inline-PTX wrappers of the block-scaled MMA path (sm_100a):
-// the kind::mxf8f6f4.block_scale instruction and its descriptor, stores into
-// TMEM, and a register fence for 32-column TMEM loads.  Single instructions,
+// the kind::mxf8f6f4.block_scale instruction and its descriptor, the shared
+// memory -> TMEM copy of scale factors (tcgen05.cp) and its descriptor, and a
+// register fence for 32-column TMEM loads.  Single instructions,
 // as in ptx.cuh; used by gemm_bs_kernel.cuh only.
 #pragma once
 
@@ -42,22 +43,43 @@ __device__ __forceinline__ void umma_f8_bs(uint32_t d_tmem, uint64_t adesc, uint
         : "memory");
 }
 
-// 32 lanes x 16 consecutive 32-bit columns: thread i of the warp writes
-// r[0..15] to columns [col, col+16) of TMEM lane (lane_base + i).
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16])
+// Copies 32 rows x 128 bits from shared memory (described by `sdesc`) into
+// TMEM lanes 0..31 of every lane quarter (the same rows in all four), columns
+// [col, col+4) of `taddr`.  Issued by one thread; ordered before the same
+// thread's later tcgen05.mma (a pipelined pair), and tracked by its
+// tcgen05.commit like an MMA.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc)
 {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// Waits for this thread's outstanding tcgen05.st.
-__device__ __forceinline__ void tmem_st_wait()
+// Shared-memory descriptor of the source of tcgen05.cp 32x128b: 32 rows of 16
+// bytes stored one after another, i.e. the K-major layout without swizzle
+// whose core matrices (8 rows x 16 bytes, 128 contiguous bytes) are 128 bytes
+// apart in the row direction (stride byte offset); one core matrix wide, so
+// the leading byte offset is unused; descriptor version 1, layout code 0 (no
+// swizzle).
+__device__ __forceinline__ uint64_t smem_desc_cp_rows16(uint32_t saddr)
 {
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
+    d |= (uint64_t)1u << 16;                           // leading byte offset (16 B, unused)
+    d |= (uint64_t)(128u >> 4) << 32;                  // stride byte offset
+    d |= (uint64_t)1u << 46;                           // version
+    return d;
+}
+
+// 16-byte shared-memory store.
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Makes this thread's generic-proxy writes to shared memory visible to the
+// async proxy (TMA, tcgen05) once ordered by a barrier.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // reg_after_wait for the 32 destination registers of a 32-column load.
