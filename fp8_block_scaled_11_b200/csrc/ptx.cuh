@@ -229,7 +229,7 @@ __device__ __forceinline__ float4 lds128(uint32_t addr)
 // CU_TENSOR_MAP_SWIZZLE_128B produces): 8-row core-matrix groups 1024 bytes
 // apart (stride byte offset), leading byte offset unused for this layout,
 // descriptor version 1 (sm_100), layout code 2 = 128-byte swizzle.
-__device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr)
+__host__ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr)
 {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
@@ -358,7 +358,7 @@ __device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t cta_m
 // wide box produces: core groups of 8 K-rows (512 bytes) are `sbo` bytes apart
 // along K; the tile is a single 64-element group along MN, so the leading
 // byte offset is not used.  Descriptor version 1, layout code 4 = 64-byte swizzle.
-__device__ __forceinline__ uint64_t smem_desc_mn_sw64(uint32_t saddr)
+__host__ __device__ __forceinline__ uint64_t smem_desc_mn_sw64(uint32_t saddr)
 {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address

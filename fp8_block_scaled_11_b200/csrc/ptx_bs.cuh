@@ -59,7 +59,7 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdes
 // apart in the row direction (stride byte offset); one core matrix wide, so
 // the leading byte offset is unused; descriptor version 1, layout code 0 (no
 // swizzle).
-__device__ __forceinline__ uint64_t smem_desc_cp_rows16(uint32_t saddr)
+__host__ __device__ __forceinline__ uint64_t smem_desc_cp_rows16(uint32_t saddr)
 {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
