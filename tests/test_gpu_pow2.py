@@ -297,3 +297,29 @@ def test_whole_k_accumulation_error_bound(K):
     rel = lambda D: np.linalg.norm(D[r].double().cpu().numpy() - ref) / np.linalg.norm(ref)
     assert rel(fast) <= (K / 32) * 2.0 ** -23, rel(fast)
     assert rel(prom) <= 1e-5, rel(prom)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("M,N,K", [(1200, 1500, 512), (256, 600, 8192)])
+def test_gemm_pow2_unaligned_output_pitch(M, N, K, dtype):
+    """Output into a view whose row pitch (N + 3 elements) is not a multiple
+    of 16 bytes, so every row is written element by element: by the block-
+    scaled kernel's epilogue (first shape: 60 tiles, no split) and by the
+    split-K reduction (second shape: 6 tiles, 64 K-blocks split).  Parity on
+    all rows; nothing written outside the view."""
+    rng = np.random.default_rng(M + N + K)
+    Kb = (K + 127) // 128
+    A = inputs.random_e4m3_bytes(M, K, seed=M)
+    B = inputs.random_e4m3_bytes(N, K, seed=N)
+    sa, sb = pow2_scales(rng, (M, Kb)), pow2_scales(rng, ((N + 127) // 128, Kb))
+    buf = torch.full((M + 1, N + 3), float("nan"), dtype=dtype, device="cuda")
+    out = buf[:M, :N]
+    ops.fp8_scaled_gemm(A.cuda(), B.cuda(), to_grid(sa), to_grid(sb), ops.SCALE_BLOCK_1x128_128x128_POW2, out=out)
+    torch.cuda.synchronize()
+    no_device_error()
+    assert torch.isnan(buf[M:]).all() and torch.isnan(buf[:M, N:]).all(), "write outside the output view"
+    ref = oracle.gemm(A.numpy(), B.numpy(), sa, sb, ops.SCALE_BLOCK_1x128_128x128)
+    if dtype == torch.float32:
+        assert_f32_close(out, ref, f"pitch N+3 M{M} N{N} K{K}")
+    else:
+        assert_bf16_close(out, ref, f"pitch N+3 M{M} N{N} K{K}")
