@@ -30,10 +30,11 @@ only the named kernel runs R times):
   quant_rows_<n>, quant_tile_<n>   the quantization sweep at n x n bf16 (n = 1024 ... 32768)
 With --time, each launch is timed with CUDA events and the mean is printed.
 
-  python profile_cases.py configs [--reps R]
+  python profile_cases.py configs [--reps R] [--graph]
 
 times every case above (the median of three rounds of R timed launches each)
-and prints one table.
+and prints one table; with --graph each round replays a CUDA graph of the R
+launches (device time, without the host's per-call work).
 """
 from __future__ import annotations
 
@@ -243,16 +244,36 @@ def _case(name):
     return _gemm_case(name) if name.startswith("gemm") else _quant_case(name)
 
 
-def _time(case, reps):
+def _time(case, reps, graph=False):
+    """Median of three rounds of `reps` back-to-back launches, ms per launch.
+    graph=True: the rounds replay a CUDA graph of the `reps` launches, so the
+    host's per-call work (argument checks, tensor-map encoding) is not in the
+    timed region -- the device-side time of launch-bound cases."""
     fn, work, unit = _case(case)
     fn()
     torch.cuda.synchronize()
+    run = fn
+    if graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        run = g.replay
     rounds = []
     for _ in range(3):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        for _ in range(reps):
-            fn()
+        if graph:
+            run()
+        else:
+            for _ in range(reps):
+                run()
         b.record()
         torch.cuda.synchronize()
         rounds.append(a.elapsed_time(b) / reps)
@@ -263,10 +284,17 @@ def _time(case, reps):
     return ms, work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9), unit
 
 
-def configs(reps):
-    print(f"{'case':22s} {'us/launch':>10s} {'rate':>10s}")
+def configs(reps, graph=False):
+    print(f"{'case':22s} {'us/launch':>10s} {'rate':>10s}" + ("  (CUDA graph)" if graph else ""))
     for case in CONFIG_CASES:
-        ms, rate, unit = _time(case, reps)
+        try:
+            ms, rate, unit = _time(case, reps, graph)
+        except RuntimeError as e:            # a launch sequence that a graph cannot capture
+            if not graph:
+                raise
+            print(f"{case:22s} {'n/a':>10s} ({str(e).splitlines()[0][:60]})")
+            torch.cuda.synchronize()
+            continue
         print(f"{case:22s} {ms * 1e3:10.1f} {rate:10.1f} {unit}")
         torch.cuda.empty_cache()
     return 0
@@ -277,9 +305,10 @@ def main(argv=None):
     ap.add_argument("case")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--time", action="store_true")
+    ap.add_argument("--graph", action="store_true", help="configs: time replays of a CUDA graph of the launches")
     a = ap.parse_args(argv)
     if a.case == "configs":
-        return configs(a.reps)
+        return configs(a.reps, a.graph)
     fn, work, unit = _case(a.case)
     fn()
     torch.cuda.synchronize()
