@@ -288,7 +288,8 @@ def run_gpu(args):
         "dtype": "e4m3 x e4m3 -> fp32 accumulate, bf16 out", "data": "synthetic (seeded N(0,1) / kaiming-uniform bf16)",
         "config": {
             "workload": "Llama4-shape FP8 linear fwd+bwd, M=16640, (N,K)=(5120,8192) and (8192,5120); "
-                        "fwd/dgrad 1x128 x 128x128, wgrad 1x128 x 1x128 (along tokens); dynamic quant included",
+                        "fwd/dgrad 1x128 x 128x128 (dgrad reads W_q as stored, MN-major), wgrad 1x128 x 1x128 "
+                        "(along tokens); dynamic quant included",
             "parallelism": f"dp{world} (independent per-GPU batches, no data-path collective)",
             "l2": "inputs larger than L2 (x alone is 272 MB); no flush",
             "vs_baseline_ref": f"pages' fp8 _scaled_mm eager fwd+bwd ({PAGES_FP8_US[0]}+{PAGES_FP8_US[1]} us, "
@@ -350,7 +351,8 @@ def gemm_roofline_list(steps, per_gemm_ms, nsteps, fp8_peak, traffic):
             tflops = 2.0 * M * N * K / (us * 1e-6) / 1e12
             key = f"{GEMM_NAMES[g]} {M}x{N}x{K}"
             out.append({"gemm": key, "recipe": recipe,
-                        "kernel": "gemm_fp8_kernel<3>" if g == 2 else "gemm_fp8_kernel<2>",
+                        "kernel": ("gemm_fp8_kernel<3>" if g == 2 else
+                                   "gemm_fp8_kernel<2>, B MN-major" if g == 1 else "gemm_fp8_kernel<2>"),
                         "bound": "tensor", "avg_launch_us": round(us, 1), "achieved": round(tflops, 1),
                         "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(tflops / fp8_peak, 3),
                         "algorithmic_bytes": gemm_algorithmic_bytes(M, N, K, recipe),
@@ -369,7 +371,7 @@ def run_ablation(args, world, dev_data, shapes, barrier, promoted_ms_step, promo
     from fp8_block_scaled_11_b200.linear import Fp8LinearStep
 
     M = inputs.LLAMA4_M
-    steps = [Fp8LinearStep(M, N, K, pow2=True) for N, K in shapes]
+    steps = [Fp8LinearStep(M, N, K, pow2=True, dgrad_wt_copy=True) for N, K in shapes]
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         for st, (x, W, dy) in zip(steps, dev_data):

@@ -37,7 +37,8 @@ struct DeviceInfo {
     bool sm100 = false;
     int num_sms = 0;
     int* err_ptr = nullptr;
-    std::atomic<bool> gemm_attr_set[16]{};   // per recipe: plain, fused output quantization, grouped
+    std::atomic<bool> gemm_attr_set[20]{};   // per instantiation: plain, fused output quantization, grouped,
+                                             // block-scaled, MN-major B
     std::atomic<int> quant_blocks[12]{};     // resident CTAs per SM, per quant kernel kind
     std::atomic<bool> tile_attr_set[16]{};   // per tile kernel kind (+8: power-of-two scale rule)
     std::atomic<int> tile_blocks[16]{};
@@ -195,15 +196,15 @@ SplitPlan plan_pair(int64_t M, int64_t N, int64_t K, int num_sms)
     return s;
 }
 
-// Which GEMM kernel a call runs: the CTA-pair kernel for an MN-major B (the
-// single-CTA kernel reads K-major operands only) and for outputs too small to
+// Which GEMM kernel a call runs: the CTA-pair kernel for outputs too small to
 // fill the GPU without splitting K (fewer, wider splits: the long-K case), the
 // single-CTA kernel otherwise (faster on large outputs, where its two 256-column
-// accumulators are fed by a single TMA ring) and for the fused output quantization.
+// accumulators are fed by a single TMA ring; K-major or MN-major B) and for the
+// fused output quantization.
 bool use_pair(int64_t M, int64_t N, int64_t K, bool b_mn, bool quant_out, int num_sms)
 {
+    (void)b_mn;
     if (quant_out) return false;
-    if (b_mn) return true;
     return plan_pair(M, N, K, num_sms).splits > 1;
 }
 
@@ -214,14 +215,14 @@ int num_sms_current()
     return d->num_sms;
 }
 
-template <int MODE, bool QOUT = false, bool GROUPED = false>
+template <int MODE, bool QOUT = false, bool GROUPED = false, bool BMN = false>
 fp8bs_status launch_gemm(DeviceInfo* d, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA,
                          const CUtensorMap& tSB,
                          const std::conditional_t<QOUT, GemmParamsQ, std::conditional_t<GROUPED, GemmParamsG, GemmParams>>& p,
                          cudaStream_t stream)
 {
-    auto k = gemm_fp8_kernel<MODE, QOUT, GROUPED>;
-    constexpr int slot = MODE + (QOUT ? 4 : 0) + (GROUPED ? 8 : 0);
+    auto k = gemm_fp8_kernel<MODE, QOUT, GROUPED, BMN>;
+    constexpr int slot = BMN ? 14 + MODE : MODE + (QOUT ? 4 : 0) + (GROUPED ? 8 : 0);
     if (!d->gemm_attr_set[slot].load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!d->gemm_attr_set[slot].load(std::memory_order_relaxed)) {
@@ -711,8 +712,12 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
     std::memset(&tSB, 0, sizeof tSB);
     if ((st = make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, lda, kBK, a_rows, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
         return st;
-    if (b_mn) {
+    if (b_mn && pair) {
         if ((st = make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, N, K, ldb, kCtaN, kStepKb * kBK, CU_TENSOR_MAP_SWIZZLE_64B)) != FP8BS_OK)
+            return st;
+    } else if (b_mn) {
+        // single-CTA kernel: K-rows x 128 N-bytes boxes, two per 256-column tile
+        if ((st = make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, N, K, ldb, kBN / 2, kBK, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK)
             return st;
     } else if ((st = make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, ldb, kBK, bt_rows, CU_TENSOR_MAP_SWIZZLE_128B)) != FP8BS_OK) {
         return st;
@@ -794,6 +799,12 @@ fp8bs_status scaled_gemm(int64_t M, int64_t N, int64_t K, const uint8_t* A, int6
     if (pow2) {
         st = mode == FP8BS_SCALE_BLOCK_1x128_128x128_POW2 ? launch_bs<kModeBlock128>(d, tA, tB, tSA, tSB, pb, stream)
                                                           : launch_bs<kModeBlock1x128>(d, tA, tB, tSA, tSB, pb, stream);
+    } else if (!pair && b_mn) {
+        switch (mode) {
+        case FP8BS_SCALE_TENSOR: st = launch_gemm<kModeTensor, false, false, true>(d, tA, tB, tSA, tSB, pb, stream); break;
+        case FP8BS_SCALE_ROWWISE: st = launch_gemm<kModeRowwise, false, false, true>(d, tA, tB, tSA, tSB, pb, stream); break;
+        default: st = launch_gemm<kModeBlock128, false, false, true>(d, tA, tB, tSA, tSB, pb, stream); break;
+        }
     } else if (!pair) {
         switch (mode) {
         case FP8BS_SCALE_TENSOR: st = launch_gemm<kModeTensor>(d, tA, tB, tSA, tSB, pb, stream); break;

@@ -205,13 +205,18 @@ __device__ __forceinline__ void decode_group_unit(const GemmParamsG& p, int64_t 
 // GROUPED: a grouped launch (GemmParamsG); 1x128 x 128x128 recipe, no split-K.
 // The tile's rows past its group's last row are multiplied with the next
 // group's rows of A (or TMA's zero fill) and never stored.
-template <int MODE, bool QOUT = false, bool GROUPED = false>
+// BMN: B given MN-major (stored K x N, N contiguous): each K-block's B tile is
+// two 128 x 128-byte boxes (K rows x N bytes, 128-byte swizzle), N-halves 16 KB
+// apart, read by the MMA through the MN-major descriptor; the 1x128 x 128x128
+// scale grid is then B's in storage order, rB(n, kb) = sb[kb + (n/128) ld_sb].
+template <int MODE, bool QOUT = false, bool GROUPED = false, bool BMN = false>
 __global__ void __launch_bounds__(EpiCfg<MODE>::threads, 1)
 gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                 const std::conditional_t<QOUT, GemmParamsQ, std::conditional_t<GROUPED, GemmParamsG, GemmParams>> p)
 {
     static_assert(!GROUPED || (MODE == kModeBlock128 && !QOUT), "grouped launches: 1x128 x 128x128, plain output");
+    static_assert(!BMN || (!GROUPED && !QOUT && MODE != kModeBlock1x128), "MN-major B: plain launches, not 1x128 x 1x128");
     using E = EpiCfg<MODE>;
     static_assert(!QOUT || E::cols == 128, "fused output quantization needs one 1x128 group per thread");
     constexpr int kEpiWarps = E::warps;
@@ -326,7 +331,13 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         if (!mbar_wait_bounded(ab_empty(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
                         mbar_arrive_expect_tx(ab_full(stage), kATileBytes + kBTileBytes);
                         tma_load_2d(sbase + SmemLayout::a_off + stage * kATileBytes, &tmA, ab_full(stage), kb * kBK, m0);
-                        tma_load_2d(sbase + SmemLayout::b_off + stage * kBTileBytes, &tmB, ab_full(stage), kb * kBK, n0);
+                        if constexpr (BMN) {
+                            const uint32_t bdst = sbase + SmemLayout::b_off + stage * kBTileBytes;
+                            tma_load_2d(bdst, &tmB, ab_full(stage), n0, kb * kBK);
+                            tma_load_2d(bdst + kBTileBytes / 2, &tmB, ab_full(stage), n0 + kBN / 2, kb * kBK);
+                        } else {
+                            tma_load_2d(sbase + SmemLayout::b_off + stage * kBTileBytes, &tmB, ab_full(stage), kb * kBK, n0);
+                        }
                         filled |= 1u << stage;
                         fill_par = (fill_par & ~(1u << stage)) | (phase << stage);
                         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -343,7 +354,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         } else if (warp == 1) {
             // ------------------------------------------------------------ MMA issuer
             if (lane == 0) {
-                constexpr uint32_t idesc = idesc_e4m3_f32(kBM, kBN);
+                constexpr uint32_t idesc = BMN ? idesc_e4m3_f32_major(kBM, kBN, 1) : idesc_e4m3_f32(kBM, kBN);
                 int stage = 0;
                 uint32_t phase = 0;
                 int tb = 0;
@@ -374,7 +385,9 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     #pragma unroll
                             for (int k = 0; k < kBK / 32; ++k) {
                                 const uint64_t adesc = smem_desc_k_sw128(a_addr + k * 32);
-                                const uint64_t bdesc = smem_desc_k_sw128(b_addr + k * 32);
+                                // MN-major: a 32-deep K step is 4 groups of 8 K-rows (4 KB)
+                                const uint64_t bdesc = BMN ? smem_desc_mn_sw128(b_addr + k * 4096, kBTileBytes / 2)
+                                                           : smem_desc_k_sw128(b_addr + k * 32);
                                 const uint32_t acc = (kPromote ? (k > 0) : (kb > kb0 || k > 0)) ? 1u : 0u;
                                 umma_f8(d_tmem, adesc, bdesc, idesc, acc);
                             }
@@ -443,7 +456,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             auto load_scales = [&](int kb, float& a, float& b) {
                 if (MODE != kModeBlock128 || kb >= kb1 || !row_ok || !nb_ok) { a = b = 0.f; return; }
                 a = __ldg(p.sa + m_glob + (int64_t)kb * p.ld_sa);
-                b = __ldg(sb_g + nb_glob + (int64_t)kb * p.ld_sb);
+                b = BMN ? __ldg(sb_g + kb + (int64_t)nb_glob * p.ld_sb) : __ldg(sb_g + nb_glob + (int64_t)kb * p.ld_sb);
             };
             float pa0, pb0, pa1, pb1;
             load_scales(kb0, pa0, pb0);

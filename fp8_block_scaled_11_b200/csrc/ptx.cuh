@@ -369,6 +369,22 @@ __host__ __device__ __forceinline__ uint64_t smem_desc_mn_sw64(uint32_t saddr)
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile stored as K rows
+// of 128 bytes (128 consecutive MN elements) with the 128-byte swizzle, in
+// chunks of 128 MN elements `chunk_bytes` apart (leading byte offset: the
+// distance between 128-element MN chunks), 8-K-row groups 1024 bytes apart
+// (stride byte offset), descriptor version 1, layout code 2 = 128-byte swizzle.
+__host__ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t chunk_bytes)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
+    d |= (uint64_t)((chunk_bytes >> 4) & 0x3FFFu) << 16;   // leading byte offset
+    d |= (uint64_t)(1024u >> 4) << 32;                 // stride byte offset: 8 K-rows x 128 B
+    d |= (uint64_t)1u << 46;                           // version
+    d |= (uint64_t)2u << 61;                           // SWIZZLE_128B
+    return d;
+}
+
 // Instruction descriptor for kind::f8f6f4 (E4M3 x E4M3 -> F32), A K-major,
 // B K-major (b_mn = 0) or MN-major (b_mn = 1).
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32_major(uint32_t M, uint32_t N, uint32_t b_mn)

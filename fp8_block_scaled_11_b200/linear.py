@@ -11,16 +11,18 @@ pytorch/ao PR #4209 (Findings So Far and review thread):
   wgrad    dW = dy^T . x    A = dy^T (1x128 along tokens),  B^T = x^T (1x128 along tokens)
 
 x: M x K, W: N x K, dy: M x N (all bf16); outputs bf16.  Three quantization
-launches per step -- x in both 1x128 directions from one read, W with its
-transposed copy, dy in both directions from one read -- and three GEMM
-launches.  With ``dgrad_wt_copy=False`` W is quantized once and dgrad reads
-the forward's W_q in its stored orientation (B MN-major, fp8_scaled_gemm_ex):
-the same result without the transposed copy, on the CTA-pair GEMM kernel.
+launches per step -- x in both 1x128 directions from one read, W 128x128, dy
+in both directions from one read -- and three GEMM launches.  dgrad reads the
+forward's W_q and scale grid in their stored orientation (B MN-major,
+fp8_scaled_gemm_ex), so W needs no transposed copy; ``dgrad_wt_copy=True``
+instead has the 128x128 launch also write the transposed bytes and grid and
+dgrad read them K-major (the same result, 42 MB more written per layer).
 With ``pow2=True`` every quantization uses the power-of-two scale rule and
 the GEMMs the matching power-of-two recipes on the block-scaled MMA (whole-K
 accumulation in TMEM, no per-K-block promotion): the fast-accumulation
 variant of pytorch/pytorch issue #159940 (Describe the bug: USE_FAST_ACCUM)
-in its B200 form, for the speed / accuracy ablation.
+in its B200 form, for the speed / accuracy ablation.  Those recipes read
+K-major operands only: pow2=True needs dgrad_wt_copy=True.
 """
 from __future__ import annotations
 
@@ -34,7 +36,7 @@ class Fp8LinearStep:
 
     LAUNCHES_PER_STEP = 6
 
-    def __init__(self, M: int, N: int, K: int, device="cuda", dgrad_wt_copy: bool = True, pow2: bool = False):
+    def __init__(self, M: int, N: int, K: int, device="cuda", dgrad_wt_copy: bool = False, pow2: bool = False):
         self.M, self.N, self.K = M, N, K
         if pow2 and not dgrad_wt_copy:
             raise ValueError("the power-of-two recipes read K-major operands only (dgrad_wt_copy=True)")

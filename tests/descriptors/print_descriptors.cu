@@ -16,6 +16,7 @@ int main()
     for (uint32_t a : addrs) {
         std::printf("smem_desc_k_sw128 %u %llu\n", a, (unsigned long long)smem_desc_k_sw128(a));
         std::printf("smem_desc_mn_sw64 %u %llu\n", a, (unsigned long long)smem_desc_mn_sw64(a));
+        std::printf("smem_desc_mn_sw128 %u %llu\n", a, (unsigned long long)smem_desc_mn_sw128(a, 16384u));
         std::printf("smem_desc_cp_rows16 %u %llu\n", a, (unsigned long long)smem_desc_cp_rows16(a));
     }
     const uint32_t shapes[][2] = {{128, 256}, {128, 128}, {128, 64}, {256, 128}, {256, 256}, {64, 8}};

@@ -16,7 +16,9 @@ the host, field by field against the descriptor tables of the PTX ISA (no GPU):
 
 The layouts the kernels need of them: K-major tiles of 128-byte rows with the
 128-byte swizzle, 8-row core-matrix groups 1024 bytes apart; the MN-major
-64-byte-swizzled B tile, 8-K-row groups 512 bytes apart; the scale-factor copy
+64-byte-swizzled B tile of the pair kernel, 8-K-row groups 512 bytes apart;
+the MN-major 128-byte-swizzled B tile of the single-CTA kernel, 8-K-row groups
+1024 bytes apart, its two 128-column halves 16 KB apart; the scale-factor copy
 source, 32 rows of 16 bytes without swizzle, 8-row core matrices 128 bytes
 apart."""
 import os
@@ -77,6 +79,17 @@ def test_k_major_128b_swizzle(values):
 def test_mn_major_64b_swizzle(values):
     for addr, v in values["smem_desc_mn_sw64"]:
         check_smem(v, addr, lbo=16, sbo=512, swizzle=4)
+
+
+def test_mn_major_128b_swizzle(values):
+    """The single-CTA kernel's MN-major B tile: K rows of 128 bytes (128 N
+    elements per swizzle atom), 8-K-row groups 1024 bytes apart (stride byte
+    offset), the two 128-column halves 16 KB apart (leading byte offset: in
+    the MN-major canonical layouts it is the step between atoms along MN)."""
+    rows = values["smem_desc_mn_sw128"]
+    assert len(rows) == 7
+    for addr, v in rows:
+        check_smem(v, addr, lbo=16384, sbo=1024, swizzle=2)
 
 
 def test_scale_factor_copy_source(values):

@@ -242,9 +242,10 @@ def test_long_k_workload(K, recipe):
 @pytest.mark.parametrize("N,K", inputs.LLAMA4_SHAPES)
 def test_llama4_fwd_bwd_workload(N, K, wt_copy):
     """The Llama4-shape linear fwd + bwd (M = 16640) at full size, in the
-    launch configuration the benchmark times (wt_copy=True) and with dgrad
-    reading W_q MN-major instead of its transposed copy; sampled output rows
-    of all three GEMMs and sampled quantized rows against the oracle."""
+    launch configuration the benchmark times (wt_copy=False: dgrad reads W_q
+    MN-major) and with dgrad reading the 128x128 kernel's transposed copy
+    instead; sampled output rows of all three GEMMs and sampled quantized rows
+    against the oracle."""
     M = inputs.LLAMA4_M
     x, W, dy = inputs.llama4(N, K)
     step = Fp8LinearStep(M, N, K, dgrad_wt_copy=wt_copy)
