@@ -434,6 +434,14 @@ def test_gemm_b_mn_major_shapes(M, N, K, mode):
     run_random_mn(M, N, K, mode, torch.bfloat16, seed=5 * M + N + K + mode)
 
 
+@pytest.mark.parametrize("mode", MN_MODES)
+def test_gemm_b_mn_major_single_cta_split_k(mode):
+    """60 output tiles, 16 K-blocks: the CTA-pair plan does not split K (too
+    many pair tiles), the single-CTA plan splits it in two, so B is read
+    MN-major by the single-CTA kernel with split-K partials and the reduction."""
+    run_random_mn(1280, 1536, 2048, mode, torch.float32, seed=17 + mode, rows=list(range(0, 1280, 37)))
+
+
 @pytest.mark.parametrize("kb", [1, 3, 64, 1001])
 def test_gemm_b_mn_major_k_blocks(kb):
     """K-block counts up to the long-K case (split-K path at 1001)."""
