@@ -1,8 +1,9 @@
 """Concurrent first use from several host threads: in a fresh process, eight
 threads start at once on their own CUDA streams and each runs the
-dual-direction quantization, the 128x128 quantization and a blockwise GEMM
-(the library's per-device set-up and per-kernel launch attributes are all
-first touched concurrently).  Every thread's results must equal the
+dual-direction quantization, the 128x128 quantization, a blockwise GEMM, the
+same GEMM reading B MN-major, and the power-of-two quantizations with the
+block-scaled GEMM (the library's per-device set-up and per-kernel launch
+attributes are all first touched concurrently).  Every thread's results must equal the
 single-threaded ones bit for bit."""
 import os
 import subprocess
@@ -25,13 +26,19 @@ build.build()
 torch.cuda.init()
 x = inputs.random_matrix(512, 1024, seed=61, dtype=torch.bfloat16).cuda()
 W = inputs.random_matrix(768, 1024, seed=62, dtype=torch.bfloat16).cuda()
+Wt = W.t().contiguous()
 torch.cuda.synchronize()
 
 def work():
     q, s, qt, st = ops.fp8_quant_1x128_dual(x)
     wq, ws, _, _ = ops.fp8_quant_128x128(W)
     y = ops.fp8_scaled_gemm(q, wq, s, ws, ops.SCALE_BLOCK_1x128_128x128, out_dtype=torch.float32)
-    return [q, s, qt, st, wq, ws, y]
+    wk, wks, _, _ = ops.fp8_quant_128x128(Wt)
+    ymn = ops.fp8_scaled_gemm_ex(q, wk, ops.MAJOR_MN, s, wks, ops.SCALE_BLOCK_1x128_128x128, out_dtype=torch.float32)
+    q2, s2 = ops.fp8_quant_1x128(x, rule=ops.SCALE_RULE_POW2)
+    w2, ws2, _, _ = ops.fp8_quant_128x128(W, rule=ops.SCALE_RULE_POW2)
+    y2 = ops.fp8_scaled_gemm(q2, w2, s2, ws2, ops.SCALE_BLOCK_1x128_128x128_POW2, out_dtype=torch.float32)
+    return [q, s, qt, st, wq, ws, y, wk, wks, ymn, q2, s2, w2, ws2, y2]
 
 results, errors = [None] * 8, []
 start = threading.Barrier(8)
